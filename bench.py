@@ -1,0 +1,411 @@
+"""Throughput benchmark of the ring attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--schedule S] [--impl reference]
+
+One step = one ``ra_ring_fwd`` call (the whole hot path: TMA tile staging, QK^T and PV on the
+tensor cores, causal masks from global positions, online softmax, partial (O, LSE) results and
+their LSE merges, the P-step ring) over the workload's synthetic inputs, resident in HBM.
+Timing: CUDA events on the launching stream around every step, L2 flushed (a 256 MiB write)
+between steps outside the events, W untimed warm-up steps, max over ranks.  N > 1 runs N
+independent replicas (one per GPU, weak scaling; the method needs no collective on one GPU).
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU fp64 oracle on the host
+cores instead (each step a bounded sample of query rows of the same workload).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s (bf16, ring P shards) and % of B200 dense BF16 peak"
+SPEC_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks sampled during the timed region (NVML reads only; no setting is changed)
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.error = repr(e)
+        self.period = period_s
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------------
+# distributed plumbing (replicas; barrier + max over ranks only)
+# ---------------------------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a scalar over all ranks (a barrier + all-reduce MAX); x itself when world == 1."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------------
+# the reference arm and the CPU baseline: the fp64 oracle on a bounded sample of rows
+# ---------------------------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleSampler:
+    """Evaluates the oracle on successive chunks of query rows of the workload (cycling heads)."""
+
+    def __init__(self, w, rows_per_step: int):
+        import numpy as np
+
+        from ring_blockwise_softmax_b200 import inputs as I
+
+        self.np = np
+        self.w = w
+        self.rows = rows_per_step
+        # Host copies of the inputs; the oracle widens the exact bf16/fp32 values to fp64.
+        q, k, v = I.make_qkv(w)
+        self.q = q.float().numpy()
+        self.k = k.float().numpy()
+        self.v = v.float().numpy()
+        self.cursor = 0
+        self.flops = 0.0
+
+    def step(self):
+        import oracle
+
+        np = self.np
+        w = self.w
+        n_heads = w.B * w.H
+        head = self.cursor % n_heads
+        start = ((self.cursor // n_heads) * self.rows * 7919) % w.N
+        self.cursor += 1
+        b, h = divmod(head, w.H)
+        rows = (start + np.arange(self.rows)) % w.N
+        pos = np.arange(w.N)
+        k = self.k[b, h].astype(np.float64)
+        v = self.v[b, h].astype(np.float64)
+        oracle.attention_rows(self.q[b, h][rows].astype(np.float64), k, v, w.scale, rows, pos, w.causal)
+        keys = (rows + 1).sum() if w.causal else self.rows * w.N
+        self.flops += 4.0 * w.d * float(keys)
+
+
+def cpu_baseline(w, budget_s: float = 12.0, rows_per_step: int = 64):
+    s = OracleSampler(w, rows_per_step)
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < budget_s:
+        s.step()
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": s.flops / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{n * rows_per_step} query rows ({rows_per_step} per chunk, cycling the {w.B * w.H} heads) of "
+                      f"the workload, fp64 numpy oracle, {dt:.1f} s"}
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    s = OracleSampler(w, args.ref_rows)
+    for _ in range(args.warmup):
+        s.step()
+    s.flops = 0.0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s.step()
+    dt = time.perf_counter() - t0
+    value = s.flops / dt / 1e12
+    cores = _blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {args.ref_rows} query rows of one head (cycling heads) of the workload"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------------------------
+def config_dict(w, args):
+    return {"workload": f"cfg{w.cfg}: {w.name}", "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "P": w.P, "layout": w.layout, "schedule": args.schedule,
+            "l2": "flushed between timed steps (256 MiB write outside the events)",
+            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+
+
+def run_gpu(args, w):
+    import torch
+
+    from ring_blockwise_softmax_b200 import inputs as I
+    from ring_blockwise_softmax_b200 import ra_attn as ra
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    peaks, peak_kind = load_peaks()
+
+    q_h, k_h, v_h = I.make_qkv(w)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    assert q.stride() == q_h.stride()
+    B, H, N, d = q.shape
+    o = torch.empty((B, H, N, d), dtype=q.dtype, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ws_bytes = ra.ring_workspace_size(q, w.P, args.schedule)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ra.ring_fwd(q, k, v, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws)
+
+    launches_per_step = 1 if (args.schedule == "fused" or w.P == 1) else w.P
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ra.get_device_status(stream) == ra.RA_OK
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_local = sum(per_step_ms) / len(per_step_ms)
+    ms = max_over_ranks(ms_local, world, dev)
+    status = ra.get_device_status(stream)
+    flops = w.flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # End to end through the public API: pinned host inputs -> device, ring forward, result -> host.
+    qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
+    qd, kd, vd = (torch.empty_strided(t.shape, t.stride(), dtype=t.dtype, device=dev) for t in (q_h, k_h, v_h))
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in (qp, kp, vp))
+    d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * lse_host.element_size()
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+
+    def e2e_step():
+        for dst, src in zip((qd, kd, vd), (qp, kp, vp)):
+            dst.copy_(src, non_blocking=True)
+        ra.ring_fwd(qd, kd, vd, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws)
+        o_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    # Standalone LSE merge of 16 fp32 partials O[1,8,16384,128] + LSE (the k-way merge kernel).
+    merge = None
+    if not args.skip_merge:
+        kparts, rows, dm = 16, 8 * 16384, 128
+        mo, ml = I.make_merge_inputs(kparts, rows, dm, seed=1104, empty_frac=0.01)
+        mo_l = [x.to(dev) for x in mo]
+        ml_l = [x.to(dev) for x in ml]
+        out_o = torch.empty(rows, dm, device=dev)
+        out_l = torch.empty(rows, device=dev)
+        for _ in range(3):
+            ra.lse_merge_n(mo_l, ml_l, out_o, out_l, stream)
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(20):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ra.lse_merge_n(mo_l, ml_l, out_o, out_l, stream)
+            b.record(stream)
+            times.append((a, b))
+        torch.cuda.synchronize()
+        mms = statistics.mean(a.elapsed_time(b) for a, b in times)
+        mbytes = (kparts + 1) * rows * (dm + 1) * 4
+        gbs = mbytes / (mms * 1e-3) / 1e9
+        merge = {"kernel": "lse_merge_n_kernel", "workload": "16 x fp32 O[1,8,16384,128] + LSE[1,8,16384]",
+                 "algorithmic_bytes": mbytes, "ms": mms, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+                 "frac": gbs / peaks["hbm_gbs"], "frac_of_8000": gbs / 8000.0}
+
+    if rank != 0:
+        return 0
+    peak = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded, shapes and distributions of the workload)",
+        "config": config_dict(w, args),
+        "pct_of_spec_bf16_peak": 100.0 * (value / world) / SPEC_BF16_TFLOPS,
+        "pct_of_measured_bf16_peak": 100.0 * (value / world) / peak,
+        "roofline": {"bound": "tensor", "kernel": "fmha_fwd_sm100", "achieved": value / world, "peak": peak,
+                     "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s", "frac": (value / world) / peak,
+                     "traffic": args.traffic,
+                     "note": "algorithmic FLOPs (4*B*H*N^2*d, halved when causal) / summed duration of the step's "
+                             f"{launches_per_step} serialised launches (CUDA events on the launch stream)"},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "device_status": ra.status_string(status),
+        "step_ms_min": min(per_step_ms), "step_ms_median": statistics.median(per_step_ms),
+    }
+    if merge is not None:
+        line["merge"] = merge
+    if not args.skip_cpu and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--schedule", choices=["stepwise", "fused"], default="fused")
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-merge", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch of the attention kernel from an ncu capture of this build")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from ring_blockwise_softmax_b200 import inputs as I
+
+    w = I.WORKLOADS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,191 @@
+/*
+ * ra_attn.h - C ABI of the B200 (sm_100a) blockwise / ring softmax attention library.
+ *
+ * What is computed (all entry points): exact softmax attention of one or more heads,
+ *
+ *     O = softmax(scale * Q K^T) V,      LSE_i = ln sum_j exp(scale * q_i . k_j),
+ *
+ * over tensors laid out as [B, H, N, d] (intelliparadigm.com, "Mosaic多轴注意力分片：突破
+ * Transformer长序列处理瓶颈", §2.1: Attention(Q,K,V) = softmax(QK^T/sqrt(d))V; intelliparadigm.com,
+ * "深度学习注意力机制优化与FlashAttention实践", §2.1).  It is computed blockwise with an online
+ * softmax: per query tile, K/V tiles stream past and a running per-row max m and sum s are
+ * updated (same FlashAttention page, §4.2; vibe-research.pages.dev, "架构层解决方案 - Sparse
+ * Attention与Ring Attention", section "Ring Attention", the blockwise identity).  A ring shard's
+ * partial result is the pair (O_partial, LSE), and two partials over disjoint key sets combine by
+ * the log-sum-exp rule LSE(a,b) = max(a,b) + log(1 + e^{-|a-b|}) (blog.gitcode.com,
+ * "分布式注意力机制突破：长序列处理的全景技术架构与实践指南", §2.2 phase 3 - printed there with
+ * the sign of the exponent wrong - and §3.4 for the M-way form).
+ *
+ * Conventions shared by every call
+ *  - Natural-log LSE of the *scaled* scores.  A query row with no visible key gets O = 0 and
+ *    LSE = -inf; merging with such a partial is the identity.
+ *  - Causal masking uses global token positions: key j is visible to query i iff
+ *    pos(j) <= pos(i).  A shard's local token t sits at global position offset + t * stride
+ *    (ra_pos_t), which covers both ring layouts: contiguous shard r = tokens [r*n, (r+1)*n);
+ *    striped shard r = tokens r, r+P, r+2P, ... (Striped Attention, git.kang-kang.com,
+ *    "注意力机制演进", timeline).
+ *  - Ownership: the caller allocates every buffer (device memory for tensor data, LSE and the
+ *    ring workspace) and every stream.  No entry point allocates device memory.
+ *  - Asynchrony: every compute call only enqueues work on the given stream(s) and returns.  The
+ *    return value reports argument and launch errors.  Faults detected on the device (a bounded
+ *    wait that ran out) are latched in a device status word read by ra_get_device_status().
+ *  - Errors never abort the process.  On a non-RA_OK return nothing has been enqueued, and
+ *    ra_last_error() returns a message for the calling thread.
+ *  - Device pointers must belong to the current CUDA device.
+ *
+ * Supported inputs
+ *  - dtype RA_BF16 (tensor-core path, fp32 accumulation, bf16 output): head dim d a multiple of 8
+ *    with d <= 128; every stride except stride[3] a multiple of 8 elements (16 bytes, TMA);
+ *    data pointer 16-byte aligned; stride[3] == 1.
+ *  - dtype RA_F32 (SIMT path, fp32 arithmetic, row sums in fp64): d <= 128, stride[3] == 1.
+ *  - B, H, N < 2^31; N of every tensor >= 1.
+ */
+#ifndef RA_ATTN_H
+#define RA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Binary-compatible with cudaStream_t / CUstream (NULL = the legacy default stream). */
+typedef struct CUstream_st* ra_stream_t;
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, mismatched tensors, bad enum value */
+  RA_ERR_UNSUPPORTED = 2,  /* valid request this build cannot run (dtype, head dim, no sm_100) */
+  RA_ERR_ALIGNMENT = 3,    /* pointer or stride violates the 16-byte rule of the bf16 path */
+  RA_ERR_WORKSPACE = 4,    /* ring workspace missing or smaller than ra_ring_workspace_size */
+  RA_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed (message in ra_last_error) */
+  RA_ERR_TIMEOUT = 6       /* a device-side bounded wait ran out (from ra_get_device_status) */
+} ra_status_t;
+
+typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype_t;
+
+typedef enum { RA_CONTIGUOUS = 0, RA_STRIPED = 1 } ra_layout_t;
+
+/* Ring schedules of ra_ring_fwd.
+ *  RA_RING_STEPWISE: P ring steps; at step t every query shard r meets KV shard (r - t) mod P in
+ *    one launch per (step, stream), and the step's partial is merged into an fp32 (O, LSE)
+ *    accumulator held in the caller's workspace by the LSE rule (the single-GPU image of P
+ *    devices each doing step t).  Pairs whose keys are all in the causal future are skipped.
+ *  RA_RING_FUSED: one launch; each query tile walks the KV shards in the same ring order and
+ *    merges each shard's partial into an on-chip accumulator with the same (m, s) rule, so no
+ *    partial result goes through HBM.  Needs no workspace. */
+typedef enum { RA_RING_STEPWISE = 0, RA_RING_FUSED = 1 } ra_ring_schedule_t;
+
+/* A strided 4-D tensor [B, H, N, d] in device memory.  stride[] is in elements (not bytes);
+ * stride[3] must be 1.  Any other strides are allowed (e.g. a head-split view of
+ * [batch, rows, features, embed] with stride[1] = head_dim and stride[2] = features*embed). */
+typedef struct {
+  void* data;
+  int32_t dtype; /* ra_dtype_t */
+  int32_t reserved;
+  int64_t shape[4];
+  int64_t stride[4];
+} ra_tensor_t;
+
+/* Global position of local token t: offset + t * stride (stride >= 1). */
+typedef struct {
+  int64_t offset;
+  int64_t stride;
+} ra_pos_t;
+
+/* Single full pass (ring with P = 1).
+ * q [B,H,Nq,d]; k, v [B,H,Nk,d]; o [B,H,Nq,d] with o->dtype == q->dtype (bf16 in -> bf16 out,
+ * fp32 in -> fp32 out); lse: fp32 [B,H,Nq] contiguous, may be NULL.  scale <= 0 selects
+ * 1/sqrt(d).  causal != 0: query i and key j both sit at position = index (0-based), key j is
+ * visible iff j <= i.  o must not overlap q, k or v. */
+ra_status_t ra_attn_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
+                        const ra_tensor_t* o, float* lse, float scale, int causal,
+                        ra_stream_t stream);
+
+/* One ring step: the partial attention of a query shard against one KV shard.
+ * k_shard, v_shard hold the shard's keys/values (any strided view, e.g. every P-th row of the
+ * full K for the striped layout).  q_pos / kv_pos give the global positions used by the causal
+ * mask (ignored when causal == 0).
+ * Output: o_part, an fp32 tensor [B,H,Nq,d] (stride[3] == 1), and lse_part, fp32 [B,H,Nq]
+ * contiguous.  O_part is normalised over the shard's visible keys.
+ * accumulate == 0: (o_part, lse_part) are overwritten with this shard's partial.
+ * accumulate != 0: (o_part, lse_part) must hold a previous partial of the same query rows over
+ *   disjoint keys; it is replaced by the LSE merge of the two (gitcode page, §2.2 phase 3).
+ * Rows whose keys are all in the future get O = 0, LSE = -inf (or are left unchanged when
+ * accumulating, since merging with an empty partial is the identity). */
+ra_status_t ra_attn_partial(const ra_tensor_t* q, const ra_tensor_t* k_shard,
+                            const ra_tensor_t* v_shard, ra_pos_t q_pos, ra_pos_t kv_pos,
+                            int causal, float scale, const ra_tensor_t* o_part, float* lse_part,
+                            int accumulate, ra_stream_t stream);
+
+/* Pairwise LSE merge of two partials of the same rows (gitcode page, §2.2 phase 3):
+ *   LSE = max(la, lb) + log1p(exp(-|la - lb|)),  O = e^{la - LSE} O_a + e^{lb - LSE} O_b.
+ * o_a, o_b, o_out: fp32 [rows, d] row-major contiguous; lse_*: fp32 [rows].  The outputs may
+ * alias either input exactly (in-place accumulate); partial overlap is not allowed.
+ * rows >= 0 (0 is a no-op), 1 <= d <= 4096.  Bound by HBM bandwidth. */
+ra_status_t ra_lse_merge(const float* o_a, const float* lse_a, const float* o_b,
+                         const float* lse_b, float* o_out, float* lse_out, int64_t rows, int d,
+                         ra_stream_t stream);
+
+/* M-way merge in one pass (gitcode page, §3.4): m = max_i LSE_i, s = sum_i e^{LSE_i - m},
+ * LSE = m + ln s, O = sum_i e^{LSE_i - m} O_i / s.
+ * o_parts, lse_parts: HOST arrays of k DEVICE pointers (read during the call only), each
+ * [rows, d] / [rows] fp32 contiguous.  1 <= k <= RA_MERGE_MAX_PARTS.  The outputs may alias
+ * o_parts[0] / lse_parts[0] exactly. */
+#define RA_MERGE_MAX_PARTS 32
+ra_status_t ra_lse_merge_n(const float* const* o_parts, const float* const* lse_parts, int k,
+                           float* o_out, float* lse_out, int64_t rows, int d,
+                           ra_stream_t stream);
+
+/* Workspace bytes ra_ring_fwd needs for (q, P, schedule): 0 for RA_RING_FUSED; for
+ * RA_RING_STEPWISE an fp32 accumulator of B*H*N*(d+1)*4 bytes (plus alignment). */
+ra_status_t ra_ring_workspace_size(const ra_tensor_t* q, int P, int schedule, size_t* bytes);
+
+/* Ring attention over P virtual sequence shards on one GPU (vibe-research page, "Ring
+ * Attention" sequence diagram; intelliparadigm.com "Mosaic…", §3.2: KV blocks rotate, Q stays,
+ * GPU r at step t uses the KV shard that started on GPU (r - t) mod P).
+ * q, k, v [B,H,N,d] of one dtype with N % P == 0; the shards are views, nothing is copied:
+ *   layout RA_CONTIGUOUS: shard r = tokens [r*N/P, (r+1)*N/P);
+ *   layout RA_STRIPED:    shard r = tokens r, r+P, r+2P, ... (token i on shard i mod P).
+ * o [B,H,N,d] (dtype of q), lse fp32 [B,H,N] contiguous (may be NULL).  Positions are the
+ * global token indices, so the result equals ra_attn_fwd(q, k, v, o, lse, scale, causal) up to
+ * rounding, for either layout.
+ * streams: n_streams >= 1 caller-owned streams (query shards are dealt round-robin over them;
+ * work for one shard stays on one stream).  The call orders itself after work already queued on
+ * streams[0] and, on return, all its work is ordered before later work on streams[0].
+ * workspace: device memory of at least ra_ring_workspace_size() bytes, 256-byte aligned (may be
+ * NULL when that size is 0).  It must not be used by other work until the call's work is done. */
+ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P,
+                        int layout, int causal, float scale, int schedule,
+                        const ra_tensor_t* o, float* lse, const ra_stream_t* streams,
+                        int n_streams, void* workspace, size_t workspace_bytes);
+
+/* Synchronises `stream`, then reads and clears the device status word that kernels set when a
+ * bounded wait runs out (each wait gives up after ra_set_wait_timeout_ns(); the kernel then
+ * stops its work, frees its tensor memory and returns, leaving its outputs undefined).
+ * Returns RA_OK, RA_ERR_TIMEOUT, or RA_ERR_CUDA if the synchronisation itself failed. */
+ra_status_t ra_get_device_status(ra_stream_t stream);
+
+/* Limit of every device-side wait, in nanoseconds (default 2e9).  Applies to later launches. */
+ra_status_t ra_set_wait_timeout_ns(uint64_t ns);
+
+/* Diagnostic: enqueue one single-CTA kernel whose threads wait on a shared-memory barrier that
+ * nothing ever arrives at, with the given limit.  The wait must give up and latch
+ * RA_ERR_TIMEOUT in the device status word; the kernel then returns normally.  Used to test the
+ * failure path without faulting or hanging the device. */
+ra_status_t ra_debug_unarrived_wait(uint64_t timeout_ns, ra_stream_t stream);
+
+const char* ra_status_string(ra_status_t status);
+
+/* Message describing the last non-RA_OK return on the calling thread ("" if none). */
+const char* ra_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int ra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RA_ATTN_H */

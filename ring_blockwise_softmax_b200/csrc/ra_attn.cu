@@ -1,0 +1,693 @@
+// ra_attn.cu - the C ABI declared in include/ra_attn.h: argument checks, TMA descriptor
+// encoding, kernel launches, the ring driver, and the device status word.
+//
+// Host code only marshals work to the kernels; every arithmetic step of the method runs on the
+// GPU.  Nothing here allocates device memory: buffers and streams come from the caller.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "../../include/ra_attn.h"
+#include "ra_attn_simt.cuh"
+#include "ra_internal.h"
+#include "ra_lse_merge.cuh"
+
+namespace ra {
+// Device status word: [0] OR of kDevStatus* flags, [1] site of the first wait that gave up.
+__device__ unsigned int g_dev_status[2];
+
+// A shared-memory barrier that nothing arrives at: the bounded wait must give up.
+__global__ void unarrived_wait_kernel(unsigned long long limit_ns, unsigned int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  WaitCtl ctl{&abort_flag, limit_ns, status};
+  (void)mbar_wait(&bar, 0, ctl, 0x901);
+}
+}  // namespace ra
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr double kLog2e = 1.4426950408889634;
+
+thread_local std::string t_last_error;
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+
+ra_status_t fail(ra_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+ra_status_t ok() {
+  t_last_error.clear();
+  return RA_OK;
+}
+
+ra_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(RA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------------------------------
+// Device / argument checks
+// ------------------------------------------------------------------------------------------
+struct DevInfo {
+  int major = -1, minor = -1, sms = 0;
+  unsigned int* status = nullptr;  // device address of ra::g_dev_status on this device
+};
+std::mutex g_dev_mu;
+DevInfo g_dev[64];
+
+ra_status_t current_device(DevInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(RA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_dev[dev].major < 0) {
+    cudaDeviceProp p;
+    e = cudaGetDeviceProperties(&p, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    g_dev[dev].major = p.major;
+    g_dev[dev].minor = p.minor;
+    g_dev[dev].sms = p.multiProcessorCount;
+    if (p.major == 10 && p.minor == 0) {
+      void* addr = nullptr;
+      e = cudaGetSymbolAddress(&addr, ra::g_dev_status);
+      if (e != cudaSuccess) {
+        g_dev[dev].major = -1;
+        return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+      }
+      g_dev[dev].status = static_cast<unsigned int*>(addr);
+    }
+  }
+  *out = g_dev[dev];
+  if (out->major != 10 || out->minor != 0)
+    return fail(RA_ERR_UNSUPPORTED, "this library is built for sm_100a (B200); device %d is sm_%d%d", dev,
+                out->major, out->minor);
+  return RA_OK;
+}
+
+const int64_t kMax32 = (int64_t(1) << 31) - 1;
+
+ra_status_t check_tensor(const ra_tensor_t* t, const char* name) {
+  if (t == nullptr) return fail(RA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (t->data == nullptr) return fail(RA_ERR_INVALID_ARG, "%s->data is NULL", name);
+  if (t->dtype != RA_F32 && t->dtype != RA_BF16) return fail(RA_ERR_INVALID_ARG, "%s->dtype %d unknown", name, t->dtype);
+  for (int i = 0; i < 4; ++i) {
+    if (t->shape[i] < 1 || t->shape[i] > kMax32)
+      return fail(RA_ERR_INVALID_ARG, "%s->shape[%d] = %lld out of range [1, 2^31)", name, i, (long long)t->shape[i]);
+    if (t->stride[i] < 0) return fail(RA_ERR_INVALID_ARG, "%s->stride[%d] is negative", name, i);
+  }
+  if (t->stride[3] != 1) return fail(RA_ERR_INVALID_ARG, "%s->stride[3] must be 1 (head dim contiguous)", name);
+  return RA_OK;
+}
+
+// The bf16 tensor-core path reads through TMA: base 16-byte aligned, strides multiples of 16 B.
+ra_status_t check_tma_tensor(const ra_tensor_t* t, const char* name) {
+  if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0)
+    return fail(RA_ERR_ALIGNMENT, "%s->data must be 16-byte aligned for the bf16 path", name);
+  for (int i = 0; i < 3; ++i)
+    if (t->shape[i] > 1 && t->stride[i] % 8 != 0)
+      return fail(RA_ERR_ALIGNMENT, "%s->stride[%d] = %lld must be a multiple of 8 elements (16 bytes)", name, i,
+                  (long long)t->stride[i]);
+  return RA_OK;
+}
+
+ra_status_t check_f32_vec_tensor(const ra_tensor_t* t, const char* name) {
+  if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0)
+    return fail(RA_ERR_ALIGNMENT, "%s->data must be 16-byte aligned", name);
+  for (int i = 0; i < 3; ++i)
+    if (t->shape[i] > 1 && t->stride[i] % 4 != 0)
+      return fail(RA_ERR_ALIGNMENT, "%s->stride[%d] must be a multiple of 4 elements", name, i);
+  return RA_OK;
+}
+
+ra_status_t check_head_dim(int d, int dtype) {
+  if (d < 1 || d > 128) return fail(RA_ERR_UNSUPPORTED, "head dim %d not in [1, 128]", d);
+  if (dtype == RA_BF16 && d % 8 != 0) return fail(RA_ERR_UNSUPPORTED, "bf16 path needs head dim %% 8 == 0 (got %d)", d);
+  return RA_OK;
+}
+
+int padded_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : 128); }
+
+float resolve_scale(float scale, int d) { return scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt((double)d)); }
+
+// ------------------------------------------------------------------------------------------
+// TMA descriptors
+// ------------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+ra_status_t get_encode(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::call_once(g_encode_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  if (g_encode == nullptr) return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorName(g_encode_err));
+  *fn = g_encode;
+  return RA_OK;
+}
+
+// 5-D view (d, token, shard, head, batch) of a bf16 tensor; strides in elements.
+struct View5 {
+  const void* base;
+  int64_t dim[5];
+  int64_t stride[5];  // stride[0] == 1
+};
+
+ra_status_t encode_view(CUtensorMap* map, const View5& v, int dp) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  ra_status_t st = get_encode(&enc);
+  if (st != RA_OK) return st;
+  cuuint64_t dims[5];
+  cuuint64_t strides[4];
+  for (int i = 0; i < 5; ++i) dims[i] = static_cast<cuuint64_t>(v.dim[i]);
+  for (int i = 1; i < 5; ++i) {
+    int64_t s = v.stride[i];
+    if (v.dim[i] == 1 || s == 0) s = 8;  // unused dimension: any valid stride
+    if (s % 8 != 0) return fail(RA_ERR_ALIGNMENT, "TMA stride %lld elements is not a multiple of 16 bytes", (long long)s);
+    strides[i - 1] = static_cast<cuuint64_t>(s) * 2;
+  }
+  const cuuint32_t box0 = dp == 32 ? 32 : 64;
+  cuuint32_t box[5] = {box0, 128, 1, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUtensorMapSwizzle swz = dp == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(v.base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return RA_OK;
+}
+
+// Shard view of a [B, H, N, d] tensor: token t of shard s is row s * shard_rows + t * tok_rows.
+View5 shard_view(const ra_tensor_t* t, int64_t n_local, int64_t P, int64_t shard_rows, int64_t tok_rows) {
+  View5 v;
+  v.base = t->data;
+  v.dim[0] = t->shape[3];
+  v.dim[1] = n_local;
+  v.dim[2] = P;
+  v.dim[3] = t->shape[1];
+  v.dim[4] = t->shape[0];
+  v.stride[0] = 1;
+  v.stride[1] = tok_rows * t->stride[2];
+  v.stride[2] = shard_rows * t->stride[2];
+  v.stride[3] = t->stride[1];
+  v.stride[4] = t->stride[0];
+  return v;
+}
+
+// ------------------------------------------------------------------------------------------
+// Launch helpers
+// ------------------------------------------------------------------------------------------
+struct Maps {
+  CUtensorMap q, k, v;
+};
+
+ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::AttnWork& w, int n_steps, int epi,
+                             cudaStream_t stream) {
+  const int B = static_cast<int>(q->shape[0]);
+  if (B > 65535 || w.H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
+  const long long gx = static_cast<long long>(w.n_q_tiles) * w.n_r;
+  if (gx > 2147483647LL) return fail(RA_ERR_UNSUPPORTED, "grid too large");
+  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(w.H), static_cast<unsigned>(B));
+  cudaError_t e;
+  if (q->dtype == RA_BF16) {
+    const int dp = padded_dim(w.d);
+    if (dp == 32)
+      e = ra::launch_fmha_dp32(maps->q, maps->k, maps->v, w, n_steps, epi, grid, stream);
+    else if (dp == 64)
+      e = ra::launch_fmha_dp64(maps->q, maps->k, maps->v, w, n_steps, epi, grid, stream);
+    else
+      e = ra::launch_fmha_dp128(maps->q, maps->k, maps->v, w, n_steps, epi, grid, stream);
+  } else {
+    const int dp = padded_dim(w.d);
+    if (dp == 32)
+      ra::attn_fwd_simt_f32<32><<<grid, 128, 0, stream>>>(w, n_steps, epi);
+    else if (dp == 64)
+      ra::attn_fwd_simt_f32<64><<<grid, 128, 0, stream>>>(w, n_steps, epi);
+    else
+      ra::attn_fwd_simt_f32<128><<<grid, 128, 0, stream>>>(w, n_steps, epi);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return RA_OK;
+}
+
+void set_operand_ptrs(ra::AttnWork& w, const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
+                      int64_t shard_rows, int64_t tok_rows) {
+  w.q = q->data;
+  w.k = k->data;
+  w.v = v->data;
+  w.q_sb = q->stride[0];
+  w.q_sh = q->stride[1];
+  w.q_rs = shard_rows * q->stride[2];
+  w.q_ts = tok_rows * q->stride[2];
+  w.k_sb = k->stride[0];
+  w.k_sh = k->stride[1];
+  w.k_rs = shard_rows * k->stride[2];
+  w.k_ts = tok_rows * k->stride[2];
+  w.v_sb = v->stride[0];
+  w.v_sh = v->stride[1];
+  w.v_rs = shard_rows * v->stride[2];
+  w.v_ts = tok_rows * v->stride[2];
+}
+
+ra_status_t check_qkv(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v) {
+  ra_status_t st;
+  if ((st = check_tensor(q, "q")) != RA_OK) return st;
+  if ((st = check_tensor(k, "k")) != RA_OK) return st;
+  if ((st = check_tensor(v, "v")) != RA_OK) return st;
+  if (k->dtype != q->dtype || v->dtype != q->dtype) return fail(RA_ERR_INVALID_ARG, "q, k, v must share one dtype");
+  if (k->shape[0] != q->shape[0] || v->shape[0] != q->shape[0] || k->shape[1] != q->shape[1] ||
+      v->shape[1] != q->shape[1])
+    return fail(RA_ERR_INVALID_ARG, "q, k, v must agree on B and H");
+  if (k->shape[3] != q->shape[3] || v->shape[3] != q->shape[3])
+    return fail(RA_ERR_INVALID_ARG, "q, k, v must share the head dim");
+  if (v->shape[2] != k->shape[2]) return fail(RA_ERR_INVALID_ARG, "k and v must have the same number of keys");
+  if ((st = check_head_dim(static_cast<int>(q->shape[3]), q->dtype)) != RA_OK) return st;
+  if (q->dtype == RA_BF16) {
+    if ((st = check_tma_tensor(q, "q")) != RA_OK) return st;
+    if ((st = check_tma_tensor(k, "k")) != RA_OK) return st;
+    if ((st = check_tma_tensor(v, "v")) != RA_OK) return st;
+  }
+  return RA_OK;
+}
+
+ra_status_t check_out(const ra_tensor_t* o, const ra_tensor_t* q, const char* name, int want_dtype) {
+  ra_status_t st = check_tensor(o, name);
+  if (st != RA_OK) return st;
+  if (o->dtype != want_dtype) return fail(RA_ERR_INVALID_ARG, "%s has the wrong dtype", name);
+  for (int i = 0; i < 4; ++i)
+    if (o->shape[i] != q->shape[i]) return fail(RA_ERR_INVALID_ARG, "%s must have the shape of q", name);
+  if (o->dtype == RA_BF16) return check_tma_tensor(o, name);
+  return RA_OK;
+}
+
+ra::AttnWork base_work(const ra_tensor_t* q, float scale, int causal, const DevInfo& dev) {
+  ra::AttnWork w{};
+  w.dev_status = dev.status;
+  w.H = static_cast<int>(q->shape[1]);
+  w.d = static_cast<int>(q->shape[3]);
+  w.causal = causal ? 1 : 0;
+  w.scale = resolve_scale(scale, w.d);
+  w.scale_log2 = static_cast<float>(static_cast<double>(w.scale) * kLog2e);
+  w.r_first = 0;
+  w.r_step = 1;
+  w.n_r = 1;
+  w.ring_step = 0;
+  w.P = 1;
+  w.wait_limit_ns = g_wait_limit_ns.load();
+  return w;
+}
+
+int q_rows_per_cta(int dtype) { return dtype == RA_BF16 ? 128 : ra::kSimtRows; }
+
+}  // namespace
+
+// ==============================================================================================
+// Entry points
+// ==============================================================================================
+extern "C" {
+
+ra_status_t ra_attn_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, const ra_tensor_t* o,
+                        float* lse, float scale, int causal, ra_stream_t stream) {
+  ra_status_t st = check_qkv(q, k, v);
+  if (st != RA_OK) return st;
+  if ((st = check_out(o, q, "o", q->dtype)) != RA_OK) return st;
+  DevInfo dev;
+  if ((st = current_device(&dev)) != RA_OK) return st;
+  ra::AttnWork w = base_work(q, scale, causal, dev);
+  w.n_q = static_cast<int>(q->shape[2]);
+  w.n_kv = static_cast<int>(k->shape[2]);
+  w.n_q_tiles = (w.n_q + q_rows_per_cta(q->dtype) - 1) / q_rows_per_cta(q->dtype);
+  w.q_off = 0;
+  w.q_rstep = 0;
+  w.q_tstride = 1;
+  w.k_off = 0;
+  w.k_sstep = 0;
+  w.k_ustride = 1;
+  set_operand_ptrs(w, q, k, v, 0, 1);
+  w.o = o->data;
+  w.o_sb = o->stride[0];
+  w.o_sh = o->stride[1];
+  w.o_rs = 0;
+  w.o_ts = o->stride[2];
+  w.lse = lse;
+  w.l_sb = q->shape[1] * q->shape[2];
+  w.l_sh = q->shape[2];
+  w.l_rs = 0;
+  w.l_ts = 1;
+
+  Maps maps;
+  if (q->dtype == RA_BF16) {
+    const int dp = padded_dim(w.d);
+    if ((st = encode_view(&maps.q, shard_view(q, w.n_q, 1, 0, 1), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.k, shard_view(k, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.v, shard_view(v, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
+  }
+  st = launch_attention(q, &maps, w, 1, ra::kEpiOut, reinterpret_cast<cudaStream_t>(stream));
+  return st == RA_OK ? ok() : st;
+}
+
+ra_status_t ra_attn_partial(const ra_tensor_t* q, const ra_tensor_t* k_shard, const ra_tensor_t* v_shard,
+                            ra_pos_t q_pos, ra_pos_t kv_pos, int causal, float scale, const ra_tensor_t* o_part,
+                            float* lse_part, int accumulate, ra_stream_t stream) {
+  ra_status_t st = check_qkv(q, k_shard, v_shard);
+  if (st != RA_OK) return st;
+  if ((st = check_out(o_part, q, "o_part", RA_F32)) != RA_OK) return st;
+  if (lse_part == nullptr) return fail(RA_ERR_INVALID_ARG, "lse_part is NULL");
+  if (q->dtype == RA_BF16 && (st = check_f32_vec_tensor(o_part, "o_part")) != RA_OK) return st;
+  if (causal && (q_pos.stride < 1 || kv_pos.stride < 1))
+    return fail(RA_ERR_INVALID_ARG, "position strides must be >= 1");
+  DevInfo dev;
+  if ((st = current_device(&dev)) != RA_OK) return st;
+  ra::AttnWork w = base_work(q, scale, causal, dev);
+  w.n_q = static_cast<int>(q->shape[2]);
+  w.n_kv = static_cast<int>(k_shard->shape[2]);
+  w.n_q_tiles = (w.n_q + q_rows_per_cta(q->dtype) - 1) / q_rows_per_cta(q->dtype);
+  w.q_off = q_pos.offset;
+  w.q_rstep = 0;
+  w.q_tstride = causal ? q_pos.stride : 1;
+  w.k_off = kv_pos.offset;
+  w.k_sstep = 0;
+  w.k_ustride = causal ? kv_pos.stride : 1;
+  set_operand_ptrs(w, q, k_shard, v_shard, 0, 1);
+  w.acc_o = static_cast<float*>(o_part->data);
+  w.a_sb = o_part->stride[0];
+  w.a_sh = o_part->stride[1];
+  w.a_rs = 0;
+  w.a_ts = o_part->stride[2];
+  w.acc_l = lse_part;
+  w.al_sb = q->shape[1] * q->shape[2];
+  w.al_sh = q->shape[2];
+  w.al_rs = 0;
+  w.al_ts = 1;
+
+  Maps maps;
+  if (q->dtype == RA_BF16) {
+    const int dp = padded_dim(w.d);
+    if ((st = encode_view(&maps.q, shard_view(q, w.n_q, 1, 0, 1), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.k, shard_view(k_shard, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.v, shard_view(v_shard, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
+  }
+  st = launch_attention(q, &maps, w, 1, accumulate ? ra::kEpiAcc : ra::kEpiPart,
+                        reinterpret_cast<cudaStream_t>(stream));
+  return st == RA_OK ? ok() : st;
+}
+
+static int merge_group(int nv) {
+  int g = 1;
+  while (g < nv && g < 32) g *= 2;
+  return g;
+}
+
+#define RA_MERGE_DISPATCH(KERNEL, VEC, G, ...)                                          \
+  switch (G) {                                                                          \
+    case 1: ra::KERNEL<VEC, 1><<<grid, 256, 0, st>>>(__VA_ARGS__); break;               \
+    case 2: ra::KERNEL<VEC, 2><<<grid, 256, 0, st>>>(__VA_ARGS__); break;               \
+    case 4: ra::KERNEL<VEC, 4><<<grid, 256, 0, st>>>(__VA_ARGS__); break;               \
+    case 8: ra::KERNEL<VEC, 8><<<grid, 256, 0, st>>>(__VA_ARGS__); break;               \
+    case 16: ra::KERNEL<VEC, 16><<<grid, 256, 0, st>>>(__VA_ARGS__); break;             \
+    default: ra::KERNEL<VEC, 32><<<grid, 256, 0, st>>>(__VA_ARGS__); break;             \
+  }
+
+static unsigned merge_grid(long long rows, int G, int sms) {
+  const long long groups_per_block = 256 / G;
+  long long blocks = (rows + groups_per_block - 1) / groups_per_block;
+  const long long cap = static_cast<long long>(sms) * 8;  // 8 blocks of 256 threads fill an SM
+  if (blocks > cap) blocks = cap;
+  return static_cast<unsigned>(blocks < 1 ? 1 : blocks);
+}
+
+static bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+ra_status_t ra_lse_merge(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b, float* o_out,
+                         float* lse_out, int64_t rows, int d, ra_stream_t stream) {
+  if (rows < 0) return fail(RA_ERR_INVALID_ARG, "rows < 0");
+  if (d < 1 || d > 4096) return fail(RA_ERR_INVALID_ARG, "d must be in [1, 4096]");
+  if (rows == 0) return ok();
+  if (!o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out) return fail(RA_ERR_INVALID_ARG, "NULL pointer");
+  DevInfo dev;
+  ra_status_t s0 = current_device(&dev);
+  if (s0 != RA_OK) return s0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool vec = d % 4 == 0 && aligned16(o_a) && aligned16(o_b) && aligned16(o_out);
+  if (vec) {
+    const int G = merge_group(d / 4);
+    dim3 grid(merge_grid(rows, G, dev.sms));
+    RA_MERGE_DISPATCH(lse_merge2_kernel, 4, G, o_a, lse_a, o_b, lse_b, o_out, lse_out, (long long)rows, d)
+  } else {
+    const int G = merge_group(d);
+    dim3 grid(merge_grid(rows, G, dev.sms));
+    RA_MERGE_DISPATCH(lse_merge2_kernel, 1, G, o_a, lse_a, o_b, lse_b, o_out, lse_out, (long long)rows, d)
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
+  return ok();
+}
+
+ra_status_t ra_lse_merge_n(const float* const* o_parts, const float* const* lse_parts, int k, float* o_out,
+                           float* lse_out, int64_t rows, int d, ra_stream_t stream) {
+  if (k < 1 || k > RA_MERGE_MAX_PARTS) return fail(RA_ERR_INVALID_ARG, "k must be in [1, %d]", RA_MERGE_MAX_PARTS);
+  if (rows < 0) return fail(RA_ERR_INVALID_ARG, "rows < 0");
+  if (d < 1 || d > 4096) return fail(RA_ERR_INVALID_ARG, "d must be in [1, 4096]");
+  if (rows == 0) return ok();
+  if (!o_parts || !lse_parts || !o_out || !lse_out) return fail(RA_ERR_INVALID_ARG, "NULL pointer");
+  ra::MergeParts parts{};
+  bool vec = d % 4 == 0 && aligned16(o_out);
+  for (int i = 0; i < k; ++i) {
+    if (!o_parts[i] || !lse_parts[i]) return fail(RA_ERR_INVALID_ARG, "NULL partial %d", i);
+    parts.o[i] = o_parts[i];
+    parts.l[i] = lse_parts[i];
+    vec = vec && aligned16(o_parts[i]);
+  }
+  DevInfo dev;
+  ra_status_t s0 = current_device(&dev);
+  if (s0 != RA_OK) return s0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (vec) {
+    const int G = merge_group(d / 4);
+    dim3 grid(merge_grid(rows, G, dev.sms));
+    RA_MERGE_DISPATCH(lse_merge_n_kernel, 4, G, parts, k, o_out, lse_out, (long long)rows, d)
+  } else {
+    const int G = merge_group(d);
+    dim3 grid(merge_grid(rows, G, dev.sms));
+    RA_MERGE_DISPATCH(lse_merge_n_kernel, 1, G, parts, k, o_out, lse_out, (long long)rows, d)
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
+  return ok();
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+ra_status_t ra_ring_workspace_size(const ra_tensor_t* q, int P, int schedule, size_t* bytes) {
+  if (bytes == nullptr) return fail(RA_ERR_INVALID_ARG, "bytes is NULL");
+  ra_status_t st = check_tensor(q, "q");
+  if (st != RA_OK) return st;
+  if (P < 1 || q->shape[2] % P != 0) return fail(RA_ERR_INVALID_ARG, "P must be >= 1 and divide N");
+  if (schedule != RA_RING_STEPWISE && schedule != RA_RING_FUSED) return fail(RA_ERR_INVALID_ARG, "unknown schedule");
+  if (schedule == RA_RING_FUSED || P == 1) {
+    *bytes = 0;
+    return ok();
+  }
+  const size_t rows = static_cast<size_t>(q->shape[0]) * q->shape[1] * q->shape[2];
+  *bytes = align256(rows * q->shape[3] * sizeof(float)) + align256(rows * sizeof(float));
+  return ok();
+}
+
+ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P, int layout,
+                        int causal, float scale, int schedule, const ra_tensor_t* o, float* lse,
+                        const ra_stream_t* streams, int n_streams, void* workspace, size_t workspace_bytes) {
+  ra_status_t st = check_qkv(q, k, v);
+  if (st != RA_OK) return st;
+  if ((st = check_out(o, q, "o", q->dtype)) != RA_OK) return st;
+  if (k->shape[2] != q->shape[2]) return fail(RA_ERR_INVALID_ARG, "ring attention needs as many keys as queries");
+  if (P < 1 || P > 64) return fail(RA_ERR_INVALID_ARG, "P must be in [1, 64]");
+  if (q->shape[2] % P != 0) return fail(RA_ERR_INVALID_ARG, "N = %lld is not a multiple of P = %d", (long long)q->shape[2], P);
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return fail(RA_ERR_INVALID_ARG, "unknown layout %d", layout);
+  if (schedule != RA_RING_STEPWISE && schedule != RA_RING_FUSED) return fail(RA_ERR_INVALID_ARG, "unknown schedule");
+  if (streams == nullptr || n_streams < 1) return fail(RA_ERR_INVALID_ARG, "need at least one stream");
+  if (n_streams > P) n_streams = P;
+  size_t need = 0;
+  if ((st = ra_ring_workspace_size(q, P, schedule, &need)) != RA_OK) return st;
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return fail(RA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  if (need > 0 && reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+    return fail(RA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  DevInfo dev;
+  if ((st = current_device(&dev)) != RA_OK) return st;
+
+  const int64_t N = q->shape[2];
+  const int64_t n_local = N / P;
+  const bool striped = layout == RA_STRIPED;
+  // Rows of shard r / local token t in the full [.., N, ..] tensors.
+  const int64_t shard_rows = striped ? 1 : n_local;
+  const int64_t tok_rows = striped ? P : 1;
+
+  ra::AttnWork w = base_work(q, scale, causal, dev);
+  w.P = P;
+  w.n_q = static_cast<int>(n_local);
+  w.n_kv = static_cast<int>(n_local);
+  w.n_q_tiles = static_cast<int>((n_local + q_rows_per_cta(q->dtype) - 1) / q_rows_per_cta(q->dtype));
+  w.q_off = 0;
+  w.q_rstep = shard_rows;
+  w.q_tstride = tok_rows;
+  w.k_off = 0;
+  w.k_sstep = shard_rows;
+  w.k_ustride = tok_rows;
+  set_operand_ptrs(w, q, k, v, shard_rows, tok_rows);
+  w.o = o->data;
+  w.o_sb = o->stride[0];
+  w.o_sh = o->stride[1];
+  w.o_rs = shard_rows * o->stride[2];
+  w.o_ts = tok_rows * o->stride[2];
+  w.lse = lse;
+  w.l_sb = q->shape[1] * N;
+  w.l_sh = N;
+  w.l_rs = shard_rows;
+  w.l_ts = tok_rows;
+  if (need > 0) {
+    const int64_t d = q->shape[3];
+    w.acc_o = static_cast<float*>(workspace);
+    w.a_ts = d;
+    w.a_rs = n_local * d;
+    w.a_sh = P * n_local * d;
+    w.a_sb = q->shape[1] * P * n_local * d;
+    const size_t o_bytes = align256(static_cast<size_t>(q->shape[0]) * q->shape[1] * N * d * sizeof(float));
+    w.acc_l = reinterpret_cast<float*>(static_cast<char*>(workspace) + o_bytes);
+    w.al_ts = 1;
+    w.al_rs = n_local;
+    w.al_sh = P * n_local;
+    w.al_sb = q->shape[1] * P * n_local;
+  }
+
+  Maps maps;
+  if (q->dtype == RA_BF16) {
+    const int dp = padded_dim(w.d);
+    if ((st = encode_view(&maps.q, shard_view(q, n_local, P, shard_rows, tok_rows), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.k, shard_view(k, n_local, P, shard_rows, tok_rows), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.v, shard_view(v, n_local, P, shard_rows, tok_rows), dp)) != RA_OK) return st;
+  }
+
+  // Fork the extra streams off streams[0] so the call is ordered after work already queued there.
+  cudaStream_t s0 = reinterpret_cast<cudaStream_t>(streams[0]);
+  cudaEvent_t ev_fork = nullptr;
+  cudaError_t e;
+  if (n_streams > 1) {
+    if ((e = cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "event");
+    if ((e = cudaEventRecord(ev_fork, s0)) != cudaSuccess) {
+      cudaEventDestroy(ev_fork);
+      return cuda_fail(e, "event record");
+    }
+    for (int i = 1; i < n_streams; ++i) {
+      if ((e = cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(streams[i]), ev_fork, 0)) != cudaSuccess) {
+        cudaEventDestroy(ev_fork);
+        return cuda_fail(e, "stream wait");
+      }
+    }
+    cudaEventDestroy(ev_fork);
+  }
+
+  st = RA_OK;
+  for (int i = 0; i < n_streams && st == RA_OK; ++i) {
+    ra::AttnWork wi = w;
+    wi.r_first = i;
+    wi.r_step = n_streams;
+    wi.n_r = (P - i + n_streams - 1) / n_streams;
+    cudaStream_t si = reinterpret_cast<cudaStream_t>(streams[i]);
+    if (schedule == RA_RING_FUSED || P == 1) {
+      wi.ring_step = 0;
+      st = launch_attention(q, &maps, wi, P, ra::kEpiOut, si);
+    } else {
+      for (int t = 0; t < P && st == RA_OK; ++t) {
+        wi.ring_step = t;
+        const int epi = t == 0 ? ra::kEpiPart : (t == P - 1 ? ra::kEpiAccOut : ra::kEpiAcc);
+        st = launch_attention(q, &maps, wi, 1, epi, si);
+      }
+    }
+  }
+
+  // Join: later work on streams[0] waits for every stream of this call.
+  for (int i = 1; i < n_streams; ++i) {
+    cudaEvent_t ev = nullptr;
+    if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "event");
+    e = cudaEventRecord(ev, reinterpret_cast<cudaStream_t>(streams[i]));
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s0, ev, 0);
+    cudaEventDestroy(ev);
+    if (e != cudaSuccess) return cuda_fail(e, "stream join");
+  }
+  return st == RA_OK ? ok() : st;
+}
+
+ra_status_t ra_get_device_status(ra_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int words[2] = {0, 0};
+  const unsigned int zero[2] = {0, 0};
+  if ((e = cudaMemcpyFromSymbol(words, ra::g_dev_status, sizeof(words))) != cudaSuccess)
+    return cuda_fail(e, "read status");
+  if (words[0] != 0) {
+    if ((e = cudaMemcpyToSymbol(ra::g_dev_status, zero, sizeof(zero))) != cudaSuccess) return cuda_fail(e, "clear");
+    if (words[0] & ra::kDevStatusTimeout)
+      return fail(RA_ERR_TIMEOUT, "a device-side wait ran out (site 0x%x)", words[1]);
+  }
+  return ok();
+}
+
+ra_status_t ra_set_wait_timeout_ns(uint64_t ns) {
+  if (ns < 1000 || ns > 60ull * 1000000000ull) return fail(RA_ERR_INVALID_ARG, "timeout must be in [1 us, 60 s]");
+  g_wait_limit_ns.store(ns);
+  return ok();
+}
+
+ra_status_t ra_debug_unarrived_wait(uint64_t timeout_ns, ra_stream_t stream) {
+  if (timeout_ns < 1000 || timeout_ns > 10ull * 1000000000ull)
+    return fail(RA_ERR_INVALID_ARG, "timeout must be in [1 us, 10 s]");
+  DevInfo dev;
+  ra_status_t st = current_device(&dev);
+  if (st != RA_OK) return st;
+  ra::unarrived_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns, dev.status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch");
+  return ok();
+}
+
+const char* ra_status_string(ra_status_t s) {
+  switch (s) {
+    case RA_OK: return "RA_OK";
+    case RA_ERR_INVALID_ARG: return "RA_ERR_INVALID_ARG";
+    case RA_ERR_UNSUPPORTED: return "RA_ERR_UNSUPPORTED";
+    case RA_ERR_ALIGNMENT: return "RA_ERR_ALIGNMENT";
+    case RA_ERR_WORKSPACE: return "RA_ERR_WORKSPACE";
+    case RA_ERR_CUDA: return "RA_ERR_CUDA";
+    case RA_ERR_TIMEOUT: return "RA_ERR_TIMEOUT";
+  }
+  return "RA_ERR_UNKNOWN";
+}
+
+const char* ra_last_error(void) { return t_last_error.c_str(); }
+
+int ra_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// ra_fmha_launch.cu - instantiates the tensor-core attention kernel for one padded head dim
+// (RA_FMHA_DP = 32, 64 or 128; the file is compiled once per value) and launches it.
+#include "ra_fmha_sm100.cuh"
+#include "ra_internal.h"
+
+#ifndef RA_FMHA_DP
+#error "compile with -DRA_FMHA_DP=32|64|128"
+#endif
+
+namespace ra {
+
+template <int EPI>
+static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
+                              int n_steps, dim3 grid, cudaStream_t stream) {
+  using C = FmhaCfg<RA_FMHA_DP>;
+  auto kern = fmha_fwd_sm100<RA_FMHA_DP, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, w, n_steps);
+  return cudaGetLastError();
+}
+
+#define RA_CAT2(a, b) a##b
+#define RA_CAT(a, b) RA_CAT2(a, b)
+
+cudaError_t RA_CAT(launch_fmha_dp, RA_FMHA_DP)(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                               const AttnWork& w, int n_steps, int epi, dim3 grid,
+                                               cudaStream_t stream) {
+  switch (epi) {
+    case kEpiOut:
+      return launch_epi<kEpiOut>(mq, mk, mv, w, n_steps, grid, stream);
+    case kEpiPart:
+      return launch_epi<kEpiPart>(mq, mk, mv, w, n_steps, grid, stream);
+    case kEpiAcc:
+      return launch_epi<kEpiAcc>(mq, mk, mv, w, n_steps, grid, stream);
+    case kEpiAccOut:
+      return launch_epi<kEpiAccOut>(mq, mk, mv, w, n_steps, grid, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace ra

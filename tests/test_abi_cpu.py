@@ -1,0 +1,98 @@
+"""CPU checks of the C ABI: the library builds, loads, exports every declared entry point, and
+rejects bad arguments on the host before touching a device.  No kernel is launched here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ra():
+    from ring_blockwise_softmax_b200 import build
+
+    build.build()
+    from ring_blockwise_softmax_b200 import ra_attn
+
+    return ra_attn
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            with open(os.path.join(ROOT, "include", fn), encoding="utf-8") as f:
+                src = f.read()
+            names.update(re.findall(r"^\s*(?:ra_status_t|const char\*|int)\s+(ra_\w+)\s*\(", src, re.M))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = _declared_symbols()
+    for want in ("ra_attn_fwd", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_fwd",
+                 "ra_ring_workspace_size", "ra_get_device_status", "ra_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(ra):
+    lib = ctypes.CDLL(ra.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(ra.SYMBOLS) == set(_declared_symbols())
+
+
+def test_status_strings_and_version(ra):
+    assert ra.status_string(ra.RA_OK) == "RA_OK"
+    assert ra.status_string(ra.RA_ERR_TIMEOUT) == "RA_ERR_TIMEOUT"
+    assert ra.version() >= 10000
+
+
+def test_host_validation_without_a_device(ra):
+    import torch
+
+    lib = ra.lib_handle()
+    # NULL tensors are rejected before any CUDA call.
+    st = lib.ra_attn_fwd(None, None, None, None, None, ctypes.c_float(0.0), 0, None)
+    assert st == ra.RA_ERR_INVALID_ARG
+    assert b"q is NULL" in lib.ra_last_error()
+    # A CPU tensor is described like any other; shape errors are found on the host.
+    q = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 3, 16, 64, dtype=torch.bfloat16)
+    tq, tk = ra.tensor_desc(q), ra.tensor_desc(k)
+    st = lib.ra_attn_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tk), ctypes.byref(tq), None,
+                         ctypes.c_float(0.0), 0, None)
+    assert st == ra.RA_ERR_INVALID_ARG and b"B and H" in lib.ra_last_error()
+    # bf16 head dim must be a multiple of 8 and <= 128
+    q2 = torch.zeros(1, 1, 16, 136, dtype=torch.bfloat16)
+    t2 = ra.tensor_desc(q2)
+    st = lib.ra_attn_fwd(ctypes.byref(t2), ctypes.byref(t2), ctypes.byref(t2), ctypes.byref(t2), None,
+                         ctypes.c_float(0.0), 0, None)
+    assert st == ra.RA_ERR_UNSUPPORTED
+    # unaligned token stride for the TMA path
+    q3 = torch.zeros(1, 1, 16, 68, dtype=torch.bfloat16)[..., :64]
+    t3 = ra.tensor_desc(q3)
+    st = lib.ra_attn_fwd(ctypes.byref(t3), ctypes.byref(t3), ctypes.byref(t3), ctypes.byref(t3), None,
+                         ctypes.c_float(0.0), 0, None)
+    assert st == ra.RA_ERR_ALIGNMENT
+    # merge with zero rows is a no-op; bad d is rejected
+    assert lib.ra_lse_merge(None, None, None, None, None, None, 0, 64, None) == ra.RA_OK
+    assert lib.ra_lse_merge(None, None, None, None, None, None, 10, 0, None) == ra.RA_ERR_INVALID_ARG
+    assert lib.ra_lse_merge_n(None, None, 0, None, None, 10, 64, None) == ra.RA_ERR_INVALID_ARG
+    assert lib.ra_lse_merge_n(None, None, 33, None, None, 10, 64, None) == ra.RA_ERR_INVALID_ARG
+    # timeout limits
+    assert lib.ra_set_wait_timeout_ns(10) == ra.RA_ERR_INVALID_ARG
+
+
+def test_ring_workspace_size(ra):
+    import torch
+
+    q = torch.zeros(2, 16, 8192, 64, dtype=torch.bfloat16)
+    assert ra.ring_workspace_size(q, 8, "fused") == 0
+    assert ra.ring_workspace_size(q, 1, "stepwise") == 0
+    rows = 2 * 16 * 8192
+    assert ra.ring_workspace_size(q, 8, "stepwise") == rows * 64 * 4 + rows * 4
+    with pytest.raises(ra.RaError):
+        ra.ring_workspace_size(q, 3, "stepwise")  # 8192 % 3 != 0
