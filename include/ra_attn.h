@@ -176,6 +176,13 @@ ra_status_t ra_set_wait_timeout_ns(uint64_t ns);
  * failure path without faulting or hanging the device. */
 ra_status_t ra_debug_unarrived_wait(uint64_t timeout_ns, ra_stream_t stream);
 
+/* Diagnostic: evaluate the two device exp2 routines of the attention kernel on n inputs (device
+ * arrays): y_poly[i] = the FMA-pipe polynomial 2^x (range reduction to [-1/2, 1/2] plus a degree-3
+ * minimax polynomial, max relative error 7.5e-5, inputs clamped at -126) and y_mufu[i] = the
+ * hardware ex2.approx.  Either output may be NULL.  Lets a test check both against their error
+ * bounds. */
+ra_status_t ra_debug_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, ra_stream_t stream);
+
 const char* ra_status_string(ra_status_t status);
 
 /* Message describing the last non-RA_OK return on the calling thread ("" if none). */

@@ -12,8 +12,9 @@
 #include <mutex>
 #include <string>
 
-#include "../../include/ra_attn.h"
+#include "ra_attn.h"
 #include "ra_attn_simt.cuh"
+#include "ra_fmha_sm100.cuh"
 #include "ra_internal.h"
 #include "ra_lse_merge.cuh"
 
@@ -33,6 +34,14 @@ __global__ void unarrived_wait_kernel(unsigned long long limit_ns, unsigned int*
   __syncthreads();
   WaitCtl ctl{&abort_flag, limit_ns, status};
   (void)mbar_wait(&bar, 0, ctl, 0x901);
+}
+__global__ void exp2_probe_kernel(const float* x, float* y_poly, float* y_mufu, long long n) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    if (y_poly) y_poly[i] = exp2_poly3(v);
+    if (y_mufu) y_mufu[i] = ex2_approx(v);
+  }
 }
 }  // namespace ra
 
@@ -224,22 +233,21 @@ struct Maps {
 };
 
 ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::AttnWork& w, int n_steps, int epi,
-                             cudaStream_t stream) {
-  const int B = static_cast<int>(q->shape[0]);
-  if (B > 65535 || w.H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
-  const long long gx = static_cast<long long>(w.n_q_tiles) * w.n_r;
-  if (gx > 2147483647LL) return fail(RA_ERR_UNSUPPORTED, "grid too large");
-  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(w.H), static_cast<unsigned>(B));
+                             int sms, cudaStream_t stream) {
+  if (w.B > 65535 || w.H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
   cudaError_t e;
   if (q->dtype == RA_BF16) {
     const int dp = padded_dim(w.d);
     if (dp == 32)
-      e = ra::launch_fmha_dp32(maps->q, maps->k, maps->v, w, n_steps, epi, grid, stream);
+      e = ra::launch_fmha_dp32(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream);
     else if (dp == 64)
-      e = ra::launch_fmha_dp64(maps->q, maps->k, maps->v, w, n_steps, epi, grid, stream);
+      e = ra::launch_fmha_dp64(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream);
     else
-      e = ra::launch_fmha_dp128(maps->q, maps->k, maps->v, w, n_steps, epi, grid, stream);
+      e = ra::launch_fmha_dp128(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream);
   } else {
+    const long long gx = static_cast<long long>(w.n_q_tiles) * w.n_r;
+    if (gx > 2147483647LL) return fail(RA_ERR_UNSUPPORTED, "grid too large");
+    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(w.H), static_cast<unsigned>(w.B));
     const int dp = padded_dim(w.d);
     if (dp == 32)
       ra::attn_fwd_simt_f32<32><<<grid, 128, 0, stream>>>(w, n_steps, epi);
@@ -306,6 +314,8 @@ ra_status_t check_out(const ra_tensor_t* o, const ra_tensor_t* q, const char* na
 ra::AttnWork base_work(const ra_tensor_t* q, float scale, int causal, const DevInfo& dev) {
   ra::AttnWork w{};
   w.dev_status = dev.status;
+  w.B = static_cast<int>(q->shape[0]);
+  w.r_major = 0;
   w.H = static_cast<int>(q->shape[1]);
   w.d = static_cast<int>(q->shape[3]);
   w.causal = causal ? 1 : 0;
@@ -365,7 +375,7 @@ ra_status_t ra_attn_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
     if ((st = encode_view(&maps.k, shard_view(k, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
     if ((st = encode_view(&maps.v, shard_view(v, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
   }
-  st = launch_attention(q, &maps, w, 1, ra::kEpiOut, reinterpret_cast<cudaStream_t>(stream));
+  st = launch_attention(q, &maps, w, 1, ra::kEpiOut, dev.sms, reinterpret_cast<cudaStream_t>(stream));
   return st == RA_OK ? ok() : st;
 }
 
@@ -410,7 +420,7 @@ ra_status_t ra_attn_partial(const ra_tensor_t* q, const ra_tensor_t* k_shard, co
     if ((st = encode_view(&maps.k, shard_view(k_shard, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
     if ((st = encode_view(&maps.v, shard_view(v_shard, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
   }
-  st = launch_attention(q, &maps, w, 1, accumulate ? ra::kEpiAcc : ra::kEpiPart,
+  st = launch_attention(q, &maps, w, 1, accumulate ? ra::kEpiAcc : ra::kEpiPart, dev.sms,
                         reinterpret_cast<cudaStream_t>(stream));
   return st == RA_OK ? ok() : st;
 }
@@ -556,6 +566,7 @@ ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
   w.k_off = 0;
   w.k_sstep = shard_rows;
   w.k_ustride = tok_rows;
+  w.r_major = striped ? 0 : 1;
   set_operand_ptrs(w, q, k, v, shard_rows, tok_rows);
   w.o = o->data;
   w.o_sb = o->stride[0];
@@ -618,12 +629,12 @@ ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
     cudaStream_t si = reinterpret_cast<cudaStream_t>(streams[i]);
     if (schedule == RA_RING_FUSED || P == 1) {
       wi.ring_step = 0;
-      st = launch_attention(q, &maps, wi, P, ra::kEpiOut, si);
+      st = launch_attention(q, &maps, wi, P, ra::kEpiOut, dev.sms, si);
     } else {
       for (int t = 0; t < P && st == RA_OK; ++t) {
         wi.ring_step = t;
         const int epi = t == 0 ? ra::kEpiPart : (t == P - 1 ? ra::kEpiAccOut : ra::kEpiAcc);
-        st = launch_attention(q, &maps, wi, 1, epi, si);
+        st = launch_attention(q, &maps, wi, 1, epi, dev.sms, si);
       }
     }
   }
@@ -668,6 +679,22 @@ ra_status_t ra_debug_unarrived_wait(uint64_t timeout_ns, ra_stream_t stream) {
   ra_status_t st = current_device(&dev);
   if (st != RA_OK) return st;
   ra::unarrived_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns, dev.status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch");
+  return ok();
+}
+
+ra_status_t ra_debug_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, ra_stream_t stream) {
+  if (n < 0) return fail(RA_ERR_INVALID_ARG, "n < 0");
+  if (n == 0) return ok();
+  if (x == nullptr) return fail(RA_ERR_INVALID_ARG, "x is NULL");
+  DevInfo dev;
+  ra_status_t st = current_device(&dev);
+  if (st != RA_OK) return st;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  ra::exp2_probe_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      x, y_poly, y_mufu, static_cast<long long>(n));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch");
   return ok();

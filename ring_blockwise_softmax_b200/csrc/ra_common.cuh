@@ -291,6 +291,8 @@ enum EpilogueMode : int {
 };
 
 struct AttnWork {
+  int B;          // batch
+  int r_major;    // work-item order: 1 = query shards outermost (contiguous shards), 0 = blocks
   int n_q;        // query tokens per shard
   int n_kv;       // key tokens per shard
   int H;          // heads

@@ -11,12 +11,16 @@ namespace ra {
 
 template <int EPI>
 static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
-                              int n_steps, dim3 grid, cudaStream_t stream) {
+                              int n_steps, int sms, cudaStream_t stream) {
   using C = FmhaCfg<RA_FMHA_DP>;
   auto kern = fmha_fwd_sm100<RA_FMHA_DP, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, w, n_steps);
+  // Persistent grid: one CTA per SM (at most one per work item of 256 query rows).
+  const long long n_items = static_cast<long long>((w.n_q + C::ROWS - 1) / C::ROWS) * w.n_r * w.H * w.B;
+  if (n_items > 2147483647LL) return cudaErrorInvalidValue;
+  const int grid = static_cast<int>(n_items < sms ? n_items : sms);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, w, n_steps, static_cast<int>(n_items));
   return cudaGetLastError();
 }
 
@@ -24,17 +28,17 @@ static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, cons
 #define RA_CAT(a, b) RA_CAT2(a, b)
 
 cudaError_t RA_CAT(launch_fmha_dp, RA_FMHA_DP)(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                               const AttnWork& w, int n_steps, int epi, dim3 grid,
+                                               const AttnWork& w, int n_steps, int epi, int sms,
                                                cudaStream_t stream) {
   switch (epi) {
     case kEpiOut:
-      return launch_epi<kEpiOut>(mq, mk, mv, w, n_steps, grid, stream);
+      return launch_epi<kEpiOut>(mq, mk, mv, w, n_steps, sms, stream);
     case kEpiPart:
-      return launch_epi<kEpiPart>(mq, mk, mv, w, n_steps, grid, stream);
+      return launch_epi<kEpiPart>(mq, mk, mv, w, n_steps, sms, stream);
     case kEpiAcc:
-      return launch_epi<kEpiAcc>(mq, mk, mv, w, n_steps, grid, stream);
+      return launch_epi<kEpiAcc>(mq, mk, mv, w, n_steps, sms, stream);
     case kEpiAccOut:
-      return launch_epi<kEpiAccOut>(mq, mk, mv, w, n_steps, grid, stream);
+      return launch_epi<kEpiAccOut>(mq, mk, mv, w, n_steps, sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

@@ -1,28 +1,33 @@
 // ra_fmha_sm100.cuh - fused blockwise attention forward on the sm_100a tensor cores.
 //
-// Computes, for one 128-row query tile, the online softmax of intelliparadigm.com
-// "深度学习注意力机制优化与FlashAttention实践" §4.2 (with the output rescaled whenever the running
-// max moves, which the printed listing omits): K/V tiles of 128 keys stream through shared
-// memory; S = Q K^T and O += P V run as tcgen05 MMAs with fp32 accumulators in tensor memory;
-// a per-row running max m and sum s are kept in fp32 registers.  One launch may walk several
-// KV shards of a ring in ring order (query shard r meets KV shard (r - t) mod P at step t,
-// vibe-research.pages.dev "Ring Attention" diagram); a shard boundary needs no extra work
-// because the running (m, s, O) already is the merged state of every shard seen so far
-// (blog.gitcode.com "分布式注意力机制突破…" §3.4: align maxima, rescale sums).
+// What it computes: the online softmax of intelliparadigm.com "深度学习注意力机制优化与
+// FlashAttention实践" §4.2 (with the output rescaled when the running max moves, which the
+// printed listing omits): K/V tiles of 128 keys stream through shared memory, S = Q K^T and
+// O += P V run as tcgen05 MMAs with fp32 accumulators in tensor memory, and a per-row running
+// max m and sum s are kept in fp32 registers.  One launch may walk several KV shards of a ring
+// in ring order (query shard r meets KV shard (r - t) mod P at step t, vibe-research.pages.dev
+// "Ring Attention" diagram); a shard boundary needs no extra work because the running
+// (m, s, O) already is the merged state of every shard seen so far (blog.gitcode.com
+// "分布式注意力机制突破…" §3.4: align the maxima, rescale the sums).
 //
-// CTA = 192 threads, one 128-row query tile:
-//   warps 0-3  softmax: thread i owns query row i = tensor-memory lane i.  Loads its S row,
-//              masks, updates (m, s), writes P (bf16) back over S in tensor memory, rescales
-//              its O row when m moved by more than 2^8 (lazy rescale; exact because the final
-//              division uses the same stale m), and runs the epilogue.
-//   warp 4     TMA producer: Q once, then K_j / V_j into a STAGES-deep ring.
-//   warp 5     MMA issuer (one thread): S_j = Q K_j^T (SS form, both K-major),
-//              O += P_j V_j (TS form: P from tensor memory, V MN-major from shared memory).
-// Tensor memory (512 columns): three S slots of 128 columns (tile j uses slot j % 3; P_j is
-// packed bf16x2 into the first 64 columns of the same slot) and O at column 384 (DP columns).
-//
-// Every wait is bounded (ra_common.cuh); on a timeout all roles stop, tensor memory is freed and
-// the kernel returns with the device status word set.
+// Structure (persistent: one CTA per SM walks work items; an item is 256 query rows = two
+// 128-row query tiles of one (batch, head, query shard); items are visited longest first):
+//   warps 0-3   softmax of query tile 0, thread i = row i = tensor-memory lane i
+//   warps 4-7   softmax of query tile 1
+//   warps 8-11  epilogue: normalise O, write O / LSE or LSE-merge into the accumulator
+//   warp 12     TMA producer: Q (two tiles) per item, then K_j / V_j into a STAGES-deep ring
+//   warp 13     MMA issuer (one thread): S_q = Q_q K_j^T (SS form), O_q += P_q V_j (TS form)
+// Both query tiles share every K/V tile (loaded once per 256 rows).  The MMA order per key
+// tile j is PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while one softmax warpgroup works on its
+// S, the tensor core runs the other tile's PV and next QK.
+// Tensor memory (512 columns): S_0, S_1 (128 fp32 columns each), O_0, O_1 (DP columns each),
+// and P_0, P_1 (bf16 pairs, 64 columns each) in their own columns when DP <= 64, otherwise over
+// the first half of S_q (then S_q is rewritten only after PV_q has consumed P_q).
+// Registers are rebalanced with setmaxnreg: softmax 168, epilogue 80, producer/MMA 96.
+// Part of the exponentials (1 in kEmuEvery columns of unmasked tiles) run as a polynomial on
+// the FMA pipe to offload the MUFU unit (exp2_poly3).
+// Every wait is bounded; on a timeout all roles stop, tensor memory is freed and the kernel
+// returns with the device status word set.
 #pragma once
 
 #include "ra_common.cuh"
@@ -32,29 +37,68 @@ namespace ra {
 template <int DP>
 struct FmhaCfg {
   static_assert(DP == 32 || DP == 64 || DP == 128, "padded head dim must be 32, 64 or 128");
-  static constexpr int BM = 128;
-  static constexpr int BN = 128;
+  static constexpr int BM = 128;    // rows of one query tile
+  static constexpr int BN = 128;    // keys of one K/V tile
+  static constexpr int ROWS = 256;  // query rows of one work item (two tiles)
   static constexpr int CB = (DP == 32) ? 32 : 64;  // columns per TMA box / swizzle span
-  static constexpr int NCB = DP / CB;              // column blocks per tile
-  static constexpr int ROW_BYTES = CB * 2;         // bytes of one row inside a column block
+  static constexpr int NCB = DP / CB;
+  static constexpr int ROW_BYTES = CB * 2;
   static constexpr uint32_t SWZ = (DP == 32) ? kSwizzle64B : kSwizzle128B;
-  static constexpr int ATOM_BYTES = 8 * ROW_BYTES;     // 8-row swizzle atom
-  static constexpr int BLOCK_BYTES = 128 * ROW_BYTES;  // one column block of a 128-row tile
-  static constexpr int TILE_BYTES = 128 * DP * 2;      // a whole Q, K or V tile (bf16)
-  static constexpr int STAGES = (DP == 128) ? 2 : (DP == 64 ? 4 : 8);  // >= 114 KB smem: one CTA per SM
-  static constexpr int NSLOT = 3;                      // S slots in tensor memory
-  static constexpr int O_COL = 384;
-  static constexpr int SMEM_TILES = TILE_BYTES * (1 + 2 * STAGES);
-  static constexpr int NBAR = 2 + 3 * STAGES + 3 * NSLOT;
-  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + SMEM_TILES + NBAR * 8 + 16 + 64 * 8;
-  static constexpr int THREADS = 192;
-  static constexpr int MAX_STEPS = 64;  // shards one launch may walk
+  static constexpr int ATOM_BYTES = 8 * ROW_BYTES;
+  static constexpr int BLOCK_BYTES = 128 * ROW_BYTES;
+  static constexpr int TILE_BYTES = 128 * DP * 2;
+  static constexpr int STAGES = (DP == 128) ? 2 : (DP == 64 ? 5 : 8);
+  static constexpr bool P_SEP = DP <= 64;
+  static constexpr int S_COL0 = 0;
+  static constexpr int O_COL0 = 256;
+  static constexpr int O_STRIDE = (DP == 128) ? 128 : 64;
+  static constexpr int P_COL0 = P_SEP ? 384 : 0;
+  static constexpr int P_STRIDE = P_SEP ? 64 : 128;
+  static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * STAGES);
+  static constexpr int NBAR = 3 + 3 * STAGES + 6 * 2;
+  static constexpr int STATS_BYTES = 2 * 128 * 8;
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES;
+  static constexpr int THREADS = 512;
+  static constexpr int D = DP;
 };
+
+#ifndef RA_REG_SOFTMAX
+#define RA_REG_SOFTMAX 168
+#endif
+#ifndef RA_REG_EPI
+#define RA_REG_EPI 80
+#endif
+#ifndef RA_REG_PROD
+#define RA_REG_PROD 96
+#endif
+static_assert(2 * 128 * RA_REG_SOFTMAX + 128 * RA_REG_EPI + 128 * RA_REG_PROD <= 65536, "register split too large");
+
+#ifndef RA_EMU_EVERY
+#define RA_EMU_EVERY 0
+#endif
+constexpr int kEmuEvery = RA_EMU_EVERY;  // 1 in kEmuEvery columns of unmasked tiles use the FMA-pipe exp2
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe: x = n + f with n = round(x) (added to the exponent field), f in
+// [-1/2, 1/2], and 2^f from a degree-3 polynomial fitted minimax in relative error by the Remez
+// exchange algorithm (max relative error 7.5e-5; coefficients from csrc/gen_exp2_poly.py).
+// Inputs below -126 are clamped, so the result is never exactly zero: callers use it only where
+// no score is masked.
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;  // 1.5 * 2^23: round(x) lands in the low mantissa bits of t
+  const float n = t - 12582912.f;
+  const float f = x - n;
+  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  // (bits(t) << 23) == n << 23 (mod 2^32): the constant part of bits(t) shifts out.
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -71,7 +115,7 @@ __device__ __forceinline__ void reg_dep(uint32_t (&r)[32]) {
                  "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 
-// Bounded wait that ignores the abort flag (used to drain in-flight TMA before exit).
+// Bounded wait that ignores the abort flag (used to drain in-flight copies / MMAs before exit).
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
@@ -79,85 +123,296 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------------------------------------
+// Work items and the walk over KV tiles
+// ---------------------------------------------------------------------------------------------
+struct Item {
+  int b, h, r, t0;
+  int rows_valid[2];
+  long long pos0;      // global position of local query token 0 of shard r
+  long long pos_last;  // position of the item's last valid query row
+};
+
+__device__ __forceinline__ void decode_item(const AttnWork& w, int idx, Item& it) {
+  const int n_blk = (w.n_q + 255) / 256;
+  const int bh_count = w.B * w.H;
+  const int bh = idx % bh_count;
+  const int rest = idx / bh_count;
+  int ri, blk;
+  if (w.r_major) {  // positions grow with the shard first (contiguous shards): longest first
+    ri = w.n_r - 1 - rest / n_blk;
+    blk = n_blk - 1 - rest % n_blk;
+  } else {
+    blk = n_blk - 1 - rest / w.n_r;
+    ri = w.n_r - 1 - rest % w.n_r;
+  }
+  it.b = bh / w.H;
+  it.h = bh % w.H;
+  it.r = w.r_first + ri * w.r_step;
+  it.t0 = blk * 256;
+  it.rows_valid[0] = max(0, min(128, w.n_q - it.t0));
+  it.rows_valid[1] = max(0, min(128, w.n_q - it.t0 - 128));
+  it.pos0 = w.q_off + static_cast<long long>(it.r) * w.q_rstep;
+  const int last = it.t0 + it.rows_valid[0] + it.rows_valid[1] - 1;
+  it.pos_last = it.pos0 + static_cast<long long>(last) * w.q_tstride;
+}
+
+struct Walk {
+  int step;  // ring step offset within this launch
+  int s;     // KV shard
+  int u0;    // first key of the current tile
+  int lim;   // keys of shard s visible to the item's last row
+};
+
+__device__ __forceinline__ bool walk_seek(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
+  for (; k.step < n_steps; ++k.step) {
+    int s = (it.r - (w.ring_step + k.step)) % w.P;
+    if (s < 0) s += w.P;
+    const int lim = visible_key_limit(w, it.pos_last, s);
+    if (lim > 0) {
+      k.s = s;
+      k.lim = lim;
+      k.u0 = 0;
+      return true;
+    }
+  }
+  return false;
+}
+
+__device__ __forceinline__ bool walk_begin(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
+  k.step = 0;
+  return walk_seek(k, w, it, n_steps);
+}
+
+__device__ __forceinline__ bool walk_next(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
+  k.u0 += FmhaCfg<32>::BN;
+  if (k.u0 < k.lim) return true;
+  ++k.step;
+  return walk_seek(k, w, it, n_steps);
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// MMA issue (single thread) and the per-row epilogue
+// ---------------------------------------------------------------------------------------------
+// Shared-memory descriptors differ only in their start-address field (bits 0-13, address >> 4),
+// so each MMA adds a small offset to a base descriptor built once.
+template <class C>
+struct DescBase {
+  uint64_t kmaj;  // K-major operand (Q, K): leading 16 B, stride = one 8-row swizzle atom
+  uint64_t vmn;   // MN-major V: leading = next 64-column block, stride = one 8-row swizzle atom
+  __device__ __forceinline__ DescBase() {
+    kmaj = make_smem_desc(0, 16, C::ATOM_BYTES, C::SWZ);
+    vmn = make_smem_desc(0, C::BLOCK_BYTES, C::ATOM_BYTES, C::SWZ);
+  }
+};
+
+__device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t saddr) {
+  return base | static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+}
+
+// S[tmem d_s] = Q (K-major, swizzled, at q_addr) * K^T (K-major at k_addr), K = D in steps of 16.
+template <class C>
+__device__ __forceinline__ void fmha_issue_qk(const DescBase<C>& db, uint32_t d_s, uint32_t q_addr, uint32_t k_addr,
+                                              uint32_t idesc) {
+  const uint64_t a0 = desc_at(db.kmaj, q_addr);
+  const uint64_t b0 = desc_at(db.kmaj, k_addr);
+#pragma unroll
+  for (int kk = 0; kk < C::D / 16; ++kk) {
+    const int cb = (kk * 16) / C::CB;
+    const uint32_t off = (cb * C::BLOCK_BYTES + ((kk * 16) % C::CB) * 2) >> 4;  // compile-time
+    mma_ss(d_s, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O[tmem d_o] (+)= P (bf16 pairs in tensor memory at p_tmem) * V (MN-major at v_addr): 16 keys
+// per MMA; the next 64-column block of V sits one BLOCK_BYTES further (leading byte offset).
+template <class C>
+__device__ __forceinline__ void fmha_issue_pv(const DescBase<C>& db, uint32_t d_o, uint32_t p_tmem, uint32_t v_addr,
+                                              uint32_t idesc, bool accumulate) {
+  const uint64_t b0 = desc_at(db.vmn, v_addr);
+#pragma unroll
+  for (int kk = 0; kk < C::BN / 16; ++kk) {
+    const uint32_t off = (kk * 16 * C::ROW_BYTES) >> 4;  // compile-time
+    mma_ts(d_o, p_tmem + kk * 8, b0 + off, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// One query row: O = O_acc / l and LSE = m ln 2 + ln l (natural log; sum_j e^{scale q.k_j} =
+// 2^m * l), then by mode: write (O bf16, LSE), write the fp32 partial, or LSE-merge it into the
+// fp32 accumulator (gitcode page §2.2 phase 3).  Warp-collective (tensor-memory loads).
+template <class C, int EPI>
+__device__ __forceinline__ void fmha_epilogue_row(const AttnWork& w, const Item& it, int t, bool row_ok,
+                                                  bool has_o, float2 ml, uint32_t o_addr) {
+  const bool has = ml.y > 0.f;
+  const float inv_l = has ? 1.f / ml.y : 0.f;
+  const float lse_part = has ? (ml.x * 0.69314718055994531f + logf(ml.y)) : -INFINITY;
+  const bool skip = (EPI == kEpiAcc) && !has;  // merging an empty partial is the identity
+  float L = lse_part, w_part = 1.f, w_acc = 0.f;
+  float* acc_row = nullptr;
+  float* accl_ptr = nullptr;
+  if (EPI != kEpiOut) {
+    acc_row = w.acc_o + it.b * w.a_sb + it.h * w.a_sh + it.r * w.a_rs + static_cast<long long>(t) * w.a_ts;
+    accl_ptr = w.acc_l + it.b * w.al_sb + it.h * w.al_sh + it.r * w.al_rs + static_cast<long long>(t) * w.al_ts;
+  }
+  if ((EPI == kEpiAcc || EPI == kEpiAccOut) && row_ok && !skip) {
+    const float la = *accl_ptr;
+    lse_merge_weights(la, lse_part, L, w_acc, w_part);
+  }
+  __nv_bfloat16* out_row = nullptr;
+  if (EPI == kEpiOut || EPI == kEpiAccOut)
+    out_row = static_cast<__nv_bfloat16*>(w.o) + it.b * w.o_sb + it.h * w.o_sh + it.r * w.o_rs +
+              static_cast<long long>(t) * w.o_ts;
+  const float wp = w_part * inv_l;
+#pragma unroll
+  for (int cc = 0; cc < C::D / 32; ++cc) {
+    uint32_t orow[32];
+    if (has_o) {
+      tmem_ld32(o_addr + cc * 32, orow);
+      tmem_ld_wait(orow);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) orow[e] = 0u;
+    }
+    if (row_ok && !skip) {
+      float vals[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) vals[e] = __uint_as_float(orow[e]) * wp;
+      if (EPI == kEpiAcc || EPI == kEpiAccOut) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          if (cc * 32 + e < w.d) {
+            const float4 a = *reinterpret_cast<const float4*>(acc_row + cc * 32 + e);
+            vals[e] = fmaf(w_acc, a.x, vals[e]);
+            vals[e + 1] = fmaf(w_acc, a.y, vals[e + 1]);
+            vals[e + 2] = fmaf(w_acc, a.z, vals[e + 2]);
+            vals[e + 3] = fmaf(w_acc, a.w, vals[e + 3]);
+          }
+        }
+      }
+      if (EPI == kEpiPart || EPI == kEpiAcc) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          if (cc * 32 + e < w.d)
+            *reinterpret_cast<float4*>(acc_row + cc * 32 + e) = make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          if (cc * 32 + e < w.d) {
+            uint4 pkt;
+            pkt.x = pack_bf16x2(vals[e], vals[e + 1]);
+            pkt.y = pack_bf16x2(vals[e + 2], vals[e + 3]);
+            pkt.z = pack_bf16x2(vals[e + 4], vals[e + 5]);
+            pkt.w = pack_bf16x2(vals[e + 6], vals[e + 7]);
+            *reinterpret_cast<uint4*>(out_row + cc * 32 + e) = pkt;
+          }
+        }
+      }
+    }
+  }
+  if (row_ok && !skip) {
+    if (EPI == kEpiPart || EPI == kEpiAcc) {
+      *accl_ptr = L;
+    } else if (w.lse != nullptr) {
+      w.lse[it.b * w.l_sb + it.h * w.l_sh + it.r * w.l_rs + static_cast<long long>(t) * w.l_ts] = L;
+    }
+  }
+}
+
+// p = 2^(s * scale_log2 - base) for the 128 scores of this row, packed to bf16 pairs and stored
+// to tensor memory; partial row sums in rsp.  EMU: 1 in kEmuEvery columns on the FMA pipe (only
+// for tiles without masked scores, see exp2_poly3).
+template <bool EMU>
+__device__ __forceinline__ void softmax_exp_store(const uint32_t (&sr)[4][32], float sl2, float base, uint32_t p_addr,
+                                                  float (&rsp)[4]) {
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float x0 = fmaf(__uint_as_float(sr[cc][2 * e]), sl2, -base);
+      const float x1 = fmaf(__uint_as_float(sr[cc][2 * e + 1]), sl2, -base);
+      const float p0 = ex2_approx(x0);
+      constexpr int kEvery = kEmuEvery > 0 ? kEmuEvery : 1;
+      const float p1 = (EMU && ((2 * e + 1) % kEvery) == kEvery - 1) ? exp2_poly3(x1) : ex2_approx(x1);
+      rsp[e & 3] += p0 + p1;
+      pk[e] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(p_addr + cc * 16, pk);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------------------------
 template <int DP, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(512, 1)
     fmha_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const AttnWork w, int n_steps) {
+                   const __grid_constant__ CUtensorMap tm_v, const AttnWork w, int n_steps, int n_items) {
   using C = FmhaCfg<DP>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
 
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::TILE_BYTES;
+  uint8_t* sQ = smem;  // two tiles
+  uint8_t* sK = sQ + 2 * C::TILE_BYTES;
   uint8_t* sV = sK + C::STAGES * C::TILE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + C::STAGES * C::TILE_BYTES);
-  uint64_t* bar_q = bars;
-  uint64_t* bar_kfull = bars + 1;
-  uint64_t* bar_vfull = bar_kfull + C::STAGES;
-  uint64_t* bar_kvempty = bar_vfull + C::STAGES;
-  uint64_t* bar_sfull = bar_kvempty + C::STAGES;
-  uint64_t* bar_pfull = bar_sfull + C::NSLOT;
-  uint64_t* bar_pvdone = bar_pfull + C::NSLOT;
-  uint64_t* bar_mma_done = bar_pvdone + C::NSLOT;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma_done + 1);
+  uint64_t* bar_q_full = bars;
+  uint64_t* bar_q_empty = bars + 1;
+  uint64_t* bar_mma_done = bars + 2;
+  uint64_t* bar_k_full = bars + 3;
+  uint64_t* bar_v_full = bar_k_full + C::STAGES;
+  uint64_t* bar_kv_empty = bar_v_full + C::STAGES;
+  uint64_t* bar_s_full = bar_kv_empty + C::STAGES;  // [2]
+  uint64_t* bar_p_full = bar_s_full + 2;            // [2]
+  uint64_t* bar_pv_done = bar_p_full + 2;           // [2]
+  uint64_t* bar_o_full = bar_pv_done + 2;           // [2]
+  uint64_t* bar_o_empty = bar_o_full + 2;           // [2]
+  uint64_t* bar_stats = bar_o_empty + 2;            // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_stats + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* walk_n = reinterpret_cast<int*>(tmem_slot + 2);
-  int* walk_shard = reinterpret_cast<int*>(tmem_slot + 4);
-  int* walk_end = walk_shard + C::MAX_STEPS;
+  float2* stats = reinterpret_cast<float2*>(tmem_slot + 4);  // [2][128] (m_used, l_sum)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  const int tile = blockIdx.x % w.n_q_tiles;
-  const int r = w.r_first + (blockIdx.x / w.n_q_tiles) * w.r_step;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int t0 = tile * C::BM;
-  const int rows_valid = min(C::BM, w.n_q - t0);
-  const long long q_pos0 = w.q_off + static_cast<long long>(r) * w.q_rstep;
-  const long long pos_last = q_pos0 + static_cast<long long>(t0 + rows_valid - 1) * w.q_tstride;
-
   WaitCtl ctl{abort_flag, w.wait_limit_ns, w.dev_status};
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
-    for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(bar_kfull + i, 1);
-      mbar_init(bar_vfull + i, 1);
-      mbar_init(bar_kvempty + i, 1);
-    }
-    for (int i = 0; i < C::NSLOT; ++i) {
-      mbar_init(bar_sfull + i, 1);
-      mbar_init(bar_pfull + i, 128);
-      mbar_init(bar_pvdone + i, 1);
-    }
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_empty, 1);
     mbar_init(bar_mma_done, 1);
-    *abort_flag = 0;
-    // The KV shards this tile visits, in ring order, and how many key tiles of each are not
-    // entirely in the causal future of the tile's last row.
-    int total = 0, n = 0;
-    for (int i = 0; i < n_steps; ++i) {
-      int s = (r - (w.ring_step + i)) % w.P;
-      if (s < 0) s += w.P;
-      const int lim = visible_key_limit(w, pos_last, s);
-      const int nt = (lim + C::BN - 1) / C::BN;
-      if (nt > 0) {
-        total += nt;
-        walk_shard[n] = s;
-        walk_end[n] = total;
-        ++n;
-      }
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(bar_k_full + i, 1);
+      mbar_init(bar_v_full + i, 1);
+      mbar_init(bar_kv_empty + i, 1);
     }
-    *walk_n = n;
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(bar_s_full + q, 1);
+      mbar_init(bar_p_full + q, 128);
+      mbar_init(bar_pv_done + q, 1);
+      mbar_init(bar_o_full + q, 1);
+      mbar_init(bar_o_empty + q, 128);
+      mbar_init(bar_stats + q, 128);
+    }
+    *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_map(&tm_q);
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
   }
-  if (warp == 5) {
+  if (warp == 13) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -165,271 +420,279 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int n_walk = *walk_n;
-  const int n_tiles = n_walk > 0 ? walk_end[n_walk - 1] : 0;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_tiles > 0) {
-      int issued = 0;
-      mbar_arrive_expect_tx(bar_q, C::TILE_BYTES);
+  if (warp >= 12) {
+    setmaxnreg_dec<RA_REG_PROD>();
+    if (warp == 12 && lane == 0) {
+      // ================================================================ TMA producer
+      int it_q = 0;
+      long long g = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+        Item it;
+        decode_item(w, idx, it);
+        Walk wk;
+        bool has = walk_begin(wk, w, it, n_steps);
+        if (!has) continue;
+        if (it_q > 0 && !mbar_wait(bar_q_empty, (it_q - 1) & 1, ctl, 0x101)) break;
+        mbar_arrive_expect_tx(bar_q_full, 2 * C::TILE_BYTES);
 #pragma unroll
-      for (int cb = 0; cb < C::NCB; ++cb)
-        tma_load_5d(sQ + cb * C::BLOCK_BYTES, &tm_q, bar_q, cb * C::CB, t0, r, h, b);
-      int wi = 0, tile_base = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        while (j >= walk_end[wi]) tile_base = walk_end[wi++];
-        const int s = walk_shard[wi];
-        const int u0 = (j - tile_base) * C::BN;
-        const int st = j % C::STAGES;
-        if (j >= C::STAGES && !mbar_wait(bar_kvempty + st, ((j / C::STAGES) - 1) & 1, ctl, 0x101)) break;
-        mbar_arrive_expect_tx(bar_kfull + st, C::TILE_BYTES);
+        for (int q = 0; q < 2; ++q)
 #pragma unroll
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_5d(sK + st * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_k, bar_kfull + st, cb * C::CB, u0, s, h, b);
-        mbar_arrive_expect_tx(bar_vfull + st, C::TILE_BYTES);
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_5d(sQ + q * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_q, bar_q_full, cb * C::CB,
+                        it.t0 + 128 * q, it.r, it.h, it.b);
+        ++it_q;
+        for (; has; has = walk_next(wk, w, it, n_steps)) {
+          const int st = static_cast<int>(g % C::STAGES);
+          if (g >= C::STAGES &&
+              !mbar_wait(bar_kv_empty + st, static_cast<uint32_t>((g / C::STAGES) - 1) & 1, ctl, 0x102)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_k_full + st, C::TILE_BYTES);
 #pragma unroll
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_5d(sV + st * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_v, bar_vfull + st, cb * C::CB, u0, s, h, b);
-        issued = j + 1;
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_5d(sK + st * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_k, bar_k_full + st, cb * C::CB, wk.u0,
+                        wk.s, it.h, it.b);
+          mbar_arrive_expect_tx(bar_v_full + st, C::TILE_BYTES);
+#pragma unroll
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_5d(sV + st * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_v, bar_v_full + st, cb * C::CB, wk.u0,
+                        wk.s, it.h, it.b);
+          ++g;
+        }
       }
-      // Make sure no TMA write to shared memory is still in flight when the CTA exits.
-      mbar_drain(bar_q, 0, w.wait_limit_ns);
-      for (int j = max(0, issued - C::STAGES); j < issued; ++j) {
-        mbar_drain(bar_kfull + j % C::STAGES, (j / C::STAGES) & 1, w.wait_limit_ns);
-        mbar_drain(bar_vfull + j % C::STAGES, (j / C::STAGES) & 1, w.wait_limit_ns);
+      // No TMA write may still be in flight when the CTA exits.
+      if (it_q > 0) mbar_drain(bar_q_full, (it_q - 1) & 1, w.wait_limit_ns);
+      for (long long j = (g > C::STAGES ? g - C::STAGES : 0); j < g; ++j) {
+        mbar_drain(bar_k_full + j % C::STAGES, static_cast<uint32_t>(j / C::STAGES) & 1, w.wait_limit_ns);
+        mbar_drain(bar_v_full + j % C::STAGES, static_cast<uint32_t>(j / C::STAGES) & 1, w.wait_limit_ns);
       }
-    }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+    } else if (warp == 13 && lane == 0) {
+      // ================================================================ MMA issuer
       constexpr uint32_t idesc_qk = make_idesc_bf16(128, C::BN, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, DP, 0, 1);
       const uint32_t q_base = smem_addr(sQ);
       const uint32_t k_base = smem_addr(sK);
       const uint32_t v_base = smem_addr(sV);
-      bool ok = mbar_wait(bar_q, 0, ctl, 0x201);
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int st = j % C::STAGES;
-          const int slot = j % C::NSLOT;
-          ok = mbar_wait(bar_kfull + st, (j / C::STAGES) & 1, ctl, 0x202);
-          if (ok && j >= C::NSLOT) ok = mbar_wait(bar_pvdone + slot, ((j - C::NSLOT) / C::NSLOT) & 1, ctl, 0x203);
+      const DescBase<C> db;
+      int it_all = 0, it_q = 0;
+      long long g = 0;
+      int c[2] = {0, 0};  // PVs issued per query tile (all items)
+      bool ok = true;
+      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+        Item it;
+        decode_item(w, idx, it);
+        Walk wk;
+        const bool has = walk_begin(wk, w, it, n_steps);
+        if (has) {
+          ok = mbar_wait(bar_q_full, it_q & 1, ctl, 0x201);
+          if (ok) ok = mbar_wait(bar_k_full + g % C::STAGES, static_cast<uint32_t>(g / C::STAGES) & 1, ctl, 0x202);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t d_s = tmem + slot * 128;
-#pragma unroll
-          for (int kk = 0; kk < DP / 16; ++kk) {
-            const int cb = (kk * 16) / C::CB;
-            const uint32_t koff = ((kk * 16) % C::CB) * 2;
-            const uint64_t a = make_smem_desc(q_base + cb * C::BLOCK_BYTES + koff, 16, C::ATOM_BYTES, C::SWZ);
-            const uint64_t bd =
-                make_smem_desc(k_base + st * C::TILE_BYTES + cb * C::BLOCK_BYTES + koff, 16, C::ATOM_BYTES, C::SWZ);
-            mma_ss(d_s, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          for (int q = 0; q < 2 && ok; ++q) {
+            // S_q may be rewritten once the previous PV_q has consumed P_q (aliased layout).
+            if (!C::P_SEP && c[q] > 0) ok = mbar_wait(bar_pv_done + q, (c[q] - 1) & 1, ctl, 0x203);
+            if (!ok) break;
+            tc_fence_after();
+            fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
+                             k_base + static_cast<int>(g % C::STAGES) * C::TILE_BYTES, idesc_qk);
+            mma_commit(bar_s_full + q);
           }
-          mma_commit(bar_sfull + slot);
-        }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int st = jj % C::STAGES;
-          const int slot = jj % C::NSLOT;
-          ok = mbar_wait(bar_pfull + slot, (jj / C::NSLOT) & 1, ctl, 0x204);
-          if (ok) ok = mbar_wait(bar_vfull + st, (jj / C::STAGES) & 1, ctl, 0x205);
           if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk) {
-            const uint32_t a_tmem = tmem + slot * 128 + kk * 8;
-            const uint64_t bd = make_smem_desc(v_base + st * C::TILE_BYTES + kk * 16 * C::ROW_BYTES, C::BLOCK_BYTES,
-                                               C::ATOM_BYTES, C::SWZ);
-            mma_ts(tmem + C::O_COL, a_tmem, bd, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+          int j = 0;
+          while (true) {
+            const long long gj = g + j;
+            const int st = static_cast<int>(gj % C::STAGES);
+            Walk nx = wk;
+            const bool has_next = walk_next(nx, w, it, n_steps);
+            if (!has_next) mma_commit(bar_q_empty);  // every QK of this item has been issued
+            for (int q = 0; q < 2 && ok; ++q) {
+              ok = mbar_wait(bar_p_full + q, c[q] & 1, ctl, 0x204);
+              if (ok && q == 0)
+                ok = mbar_wait(bar_v_full + st, static_cast<uint32_t>(gj / C::STAGES) & 1, ctl, 0x205);
+              if (ok && j == 0 && it_all > 0) ok = mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x206);
+              if (!ok) break;
+              tc_fence_after();
+              fmha_issue_pv<C>(db, tmem + C::O_COL0 + C::O_STRIDE * q, tmem + C::P_COL0 + C::P_STRIDE * q,
+                               v_base + st * C::TILE_BYTES, idesc_pv, j > 0);
+              mma_commit(bar_pv_done + q);
+              ++c[q];
+              if (has_next) {
+                const long long gn = gj + 1;
+                if (q == 0)
+                  ok = mbar_wait(bar_k_full + gn % C::STAGES, static_cast<uint32_t>(gn / C::STAGES) & 1, ctl, 0x207);
+                if (ok && !C::P_SEP) ok = mbar_wait(bar_pv_done + q, (c[q] - 1) & 1, ctl, 0x208);
+                if (!ok) break;
+                tc_fence_after();
+                fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
+                                 k_base + static_cast<int>(gn % C::STAGES) * C::TILE_BYTES, idesc_qk);
+                mma_commit(bar_s_full + q);
+              }
+            }
+            if (!ok) break;
+            mma_commit(bar_kv_empty + st);
+            ++j;
+            if (!has_next) break;
+            wk = nx;
           }
-          mma_commit(bar_pvdone + slot);
-          mma_commit(bar_kvempty + st);
+          if (!ok) break;
+          g += j;
+          ++it_q;
         }
+        if (!has && it_all > 0) {
+          // An item with no visible key issues no PV; still keep o_full at most one phase ahead
+          // of the epilogue warps, which wait on it by parity.
+          for (int q = 0; q < 2 && ok; ++q) ok = mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x209);
+          if (!ok) break;
+        }
+        mma_commit(bar_o_full + 0);
+        mma_commit(bar_o_full + 1);
+        ++it_all;
       }
-      // Tensor memory is freed below only after every MMA issued here has completed.
+      // Tensor memory is freed only after every MMA issued here has completed.
       mma_commit(bar_mma_done);
       mbar_drain(bar_mma_done, 0, w.wait_limit_ns);
     }
-  } else {
-    // ------------------------------------------------------------------ softmax + epilogue
-    const int row = threadIdx.x;  // 0..127 == tensor-memory lane
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const bool row_ok = row < rows_valid;
-    const long long pos_q = q_pos0 + static_cast<long long>(t0 + row) * w.q_tstride;
+  } else if (warp < 8) {
+    setmaxnreg_inc<RA_REG_SOFTMAX>();
+    // ================================================================ softmax (query tile q)
+    const int q = warp >> 2;
+    const int row = threadIdx.x & 127;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_addr = lane_addr + C::S_COL0 + 128 * q;
+    const uint32_t p_addr = lane_addr + C::P_COL0 + C::P_STRIDE * q;
+    const uint32_t o_addr = lane_addr + C::O_COL0 + C::O_STRIDE * q;
     const float sl2 = w.scale_log2;
-    float m_used = -INFINITY;  // running max of scaled scores, log2 units
-    float l_sum = 0.f;         // running sum of 2^(x - m_used)
+    int it_all = 0, c = 0;
     bool ok = true;
-    int wi = 0, tile_base = 0;
-    int row_lim = (n_tiles > 0 && row_ok) ? visible_key_limit(w, pos_q, walk_shard[0]) : w.n_kv;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (j >= walk_end[wi]) {
-        tile_base = walk_end[wi++];
-        row_lim = row_ok ? visible_key_limit(w, pos_q, walk_shard[wi]) : w.n_kv;
-      }
-      const int slot = j % C::NSLOT;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull + slot, (j / C::NSLOT) & 1, ctl, 0x301));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + slot * 128 + c * 32, sr[c]);
-      tmem_ld_wait(sr[0]);
-      reg_dep(sr[1]);
-      reg_dep(sr[2]);
-      reg_dep(sr[3]);
-
-      const int lim = row_lim - (j - tile_base) * C::BN;  // keys [0, lim) of this tile are visible
-      if (lim < C::BN) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c >> 5][c & 31]));
-      const float m_tile = mx * sl2;
-      float m_new = m_used;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (m_tile > m_used) {
-        if (m_used == -INFINITY) {
-          m_new = m_tile;  // nothing accumulated yet: this row of O is still zero
-        } else if (m_tile > m_used + 8.f) {
-          m_new = m_tile;
-          alpha = ex2_approx(m_used - m_new);
-          rescale = true;
+    for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+      Item it;
+      decode_item(w, idx, it);
+      const bool row_ok = row < it.rows_valid[q];
+      const long long pos_q = it.pos0 + static_cast<long long>(it.t0 + 128 * q + row) * w.q_tstride;
+      float m_used = -INFINITY;  // running max of scaled scores, log2 units
+      float l_sum = 0.f;         // running sum of 2^(x - m_used)
+      Walk wk;
+      int cur_s = -1, row_lim = 0;
+      for (bool has = walk_begin(wk, w, it, n_steps); has; has = walk_next(wk, w, it, n_steps)) {
+        if (wk.s != cur_s) {
+          cur_s = wk.s;
+          row_lim = row_ok ? visible_key_limit(w, pos_q, wk.s) : w.n_kv;
         }
-      }
-      const float base = (m_new == -INFINITY) ? 0.f : m_new;
-      float rs = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]), sl2, -base));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]), sl2, -base));
-        rs += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O holds sum_{i<j} P_i V_i only once PV_{j-1} has completed.
-        const int jp = j - 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone + jp % C::NSLOT, (jp / C::NSLOT) & 1, ctl, 0x302));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + q, c & 1, ctl, 0x301));
         if (!ok) break;
         tc_fence_after();
+        uint32_t sr[4][32];
 #pragma unroll
-        for (int c = 0; c < DP / 32; ++c) {
-          uint32_t orow[32];
-          tmem_ld32(lane_addr + C::O_COL + c * 32, orow);
-          tmem_ld_wait(orow);
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_addr + cc * 32, sr[cc]);
+        tmem_ld_wait(sr[0]);
+        reg_dep(sr[1]);
+        reg_dep(sr[2]);
+        reg_dep(sr[3]);
+        const int lim = row_lim - wk.u0;  // keys [0, lim) of this tile are visible to this row
+        const bool masked = __any_sync(0xffffffffu, lim < C::BN);
+        if (lim < C::BN) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
-          tmem_st32(lane_addr + C::O_COL + c * 32, orow);
+          for (int e = 0; e < 128; ++e)
+            if (e >= lim) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
         }
-      }
-      l_sum = l_sum * alpha + rs;
-      m_used = m_new;
-      tmem_st16(lane_addr + slot * 128, pk);
-      tmem_st16(lane_addr + slot * 128 + 16, pk + 16);
-      tmem_st16(lane_addr + slot * 128 + 32, pk + 32);
-      tmem_st16(lane_addr + slot * 128 + 48, pk + 48);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar_pfull + slot);
-    }
-
-    // ---------------------------------------------------------------- epilogue
-    // Merging with an empty partial is the identity: nothing to read or write.
-    if (EPI == kEpiAcc && n_tiles == 0) ok = false;
-    if (ok && n_tiles > 0) {
-      const int jl = n_tiles - 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone + jl % C::NSLOT, (jl / C::NSLOT) & 1, ctl, 0x303));
-      if (ok) tc_fence_after();
-    }
-    if (ok) {
-      const bool has = l_sum > 0.f;
-      const float inv_l = has ? 1.f / l_sum : 0.f;
-      // LSE in natural log: sum_j e^{scale q.k_j} = 2^{m_used} * l_sum.
-      const float lse_part = has ? (m_used * 0.69314718055994531f + logf(l_sum)) : -INFINITY;
-      float L = lse_part, w_part = 1.f, w_acc = 0.f;
-      float* acc_row = nullptr;
-      if (EPI == kEpiPart || EPI == kEpiAcc || EPI == kEpiAccOut) {
-        acc_row = w.acc_o + b * w.a_sb + h * w.a_sh + r * w.a_rs + static_cast<long long>(t0 + row) * w.a_ts;
-      }
-      float* accl_ptr = nullptr;
-      if (EPI != kEpiOut)
-        accl_ptr = w.acc_l + b * w.al_sb + h * w.al_sh + r * w.al_rs + static_cast<long long>(t0 + row) * w.al_ts;
-      if ((EPI == kEpiAcc || EPI == kEpiAccOut) && row_ok) {
-        const float la = *accl_ptr;
-        lse_merge_weights(la, lse_part, L, w_acc, w_part);
-      }
-      __nv_bfloat16* out_row = nullptr;
-      if (EPI == kEpiOut || EPI == kEpiAccOut)
-        out_row = static_cast<__nv_bfloat16*>(w.o) + b * w.o_sb + h * w.o_sh + r * w.o_rs +
-                  static_cast<long long>(t0 + row) * w.o_ts;
-      const float wp = w_part * inv_l;
+        // Row max as 8 independent chains (a single chain of 128 dependent max operations would
+        // be latency-bound).
+        float mxp[8];
 #pragma unroll
-      for (int c = 0; c < DP / 32; ++c) {
-        uint32_t orow[32];
-        if (n_tiles > 0) {
-          tmem_ld32(lane_addr + C::O_COL + c * 32, orow);
-          tmem_ld_wait(orow);
-        } else {
+        for (int i = 0; i < 8; ++i) mxp[i] = __uint_as_float(sr[0][i]);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orow[e] = 0u;
-        }
-        if (row_ok) {
-          float vals[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) vals[e] = __uint_as_float(orow[e]) * wp;
-          if (EPI == kEpiAcc || EPI == kEpiAccOut) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              if (c * 32 + e < w.d) {
-                const float4 a = *reinterpret_cast<const float4*>(acc_row + c * 32 + e);
-                vals[e] = fmaf(w_acc, a.x, vals[e]);
-                vals[e + 1] = fmaf(w_acc, a.y, vals[e + 1]);
-                vals[e + 2] = fmaf(w_acc, a.z, vals[e + 2]);
-                vals[e + 3] = fmaf(w_acc, a.w, vals[e + 3]);
-              }
-            }
-          }
-          if (EPI == kEpiPart || EPI == kEpiAcc) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              if (c * 32 + e < w.d)
-                *reinterpret_cast<float4*>(acc_row + c * 32 + e) =
-                    make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              if (c * 32 + e < w.d) {
-                uint4 pkt;
-                pkt.x = pack_bf16x2(vals[e], vals[e + 1]);
-                pkt.y = pack_bf16x2(vals[e + 2], vals[e + 3]);
-                pkt.z = pack_bf16x2(vals[e + 4], vals[e + 5]);
-                pkt.w = pack_bf16x2(vals[e + 6], vals[e + 7]);
-                *reinterpret_cast<uint4*>(out_row + c * 32 + e) = pkt;
-              }
-            }
+        for (int e = 8; e < 128; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], __uint_as_float(sr[e >> 5][e & 31]));
+        const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                               fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        const float m_tile = mx * sl2;
+        float m_new = m_used;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m_tile > m_used) {
+          if (m_used == -INFINITY) {
+            m_new = m_tile;  // nothing accumulated yet in this item: this row of O is zero
+          } else if (m_tile > m_used + 8.f) {
+            m_new = m_tile;
+            alpha = ex2_approx(m_used - m_new);
+            rescale = true;
           }
         }
-      }
-      if (row_ok) {
-        if (EPI == kEpiPart || EPI == kEpiAcc) {
-          *accl_ptr = L;
-        } else if (w.lse != nullptr) {
-          w.lse[b * w.l_sb + h * w.l_sh + r * w.l_rs + static_cast<long long>(t0 + row) * w.l_ts] = L;
+        const float base = (m_new == -INFINITY) ? 0.f : m_new;
+        // P_q in its own columns is free once the previous PV_q has read it; the O rescale
+        // needs that PV to have landed too.
+        const bool any_rescale = __any_sync(0xffffffffu, rescale);
+        if ((C::P_SEP || any_rescale) && c > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + q, (c - 1) & 1, ctl, 0x302));
+          if (!ok) break;
+          tc_fence_after();
         }
+        float rsp[4] = {0.f, 0.f, 0.f, 0.f};  // row sum as 4 independent chains
+        if (masked || kEmuEvery == 0)
+          softmax_exp_store<false>(sr, sl2, base, p_addr, rsp);
+        else
+          softmax_exp_store<true>(sr, sl2, base, p_addr, rsp);
+        if (any_rescale) {
+#pragma unroll
+          for (int cc = 0; cc < DP / 32; ++cc) {
+            uint32_t orow[32];
+            tmem_ld32(o_addr + cc * 32, orow);
+            tmem_ld_wait(orow);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+            tmem_st32(o_addr + cc * 32, orow);
+          }
+        }
+        l_sum = l_sum * alpha + ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3]));
+        m_used = m_new;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p_full + q);
+        ++c;
       }
+      if (!ok) break;
+      // Hand (m, l) of this item to the epilogue warps once they are done with the previous item.
+      if (it_all > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x303));
+        if (!ok) break;
+      }
+      stats[q * 128 + row] = make_float2(m_used, l_sum);
+      mbar_arrive(bar_stats + q);
+      ++it_all;
+    }
+  } else {
+    setmaxnreg_dec<RA_REG_EPI>();
+    // ================================================================ epilogue (both tiles)
+    const int row = threadIdx.x & 127;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    int it_all = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+      Item it;
+      decode_item(w, idx, it);
+      Walk wk;
+      const bool has_o = walk_begin(wk, w, it, n_steps);
+      for (int q = 0; q < 2; ++q) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_full + q, it_all & 1, ctl, 0x401) &&
+                                         mbar_wait(bar_stats + q, it_all & 1, ctl, 0x402));
+        if (!ok) break;
+        tc_fence_after();
+        const float2 ml = stats[q * 128 + row];
+        const bool row_ok = row < it.rows_valid[q];
+        const int t = it.t0 + 128 * q + row;
+        fmha_epilogue_row<C, EPI>(w, it, t, row_ok, has_o, ml, lane_addr + C::O_COL0 + C::O_STRIDE * q);
+        tc_fence_before();
+        mbar_arrive(bar_o_empty + q);
+      }
+      ++it_all;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -9,10 +9,10 @@
 namespace ra {
 
 cudaError_t launch_fmha_dp32(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
-                             int n_steps, int epi, dim3 grid, cudaStream_t stream);
+                             int n_steps, int epi, int sms, cudaStream_t stream);
 cudaError_t launch_fmha_dp64(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
-                             int n_steps, int epi, dim3 grid, cudaStream_t stream);
+                             int n_steps, int epi, int sms, cudaStream_t stream);
 cudaError_t launch_fmha_dp128(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
-                              int n_steps, int epi, dim3 grid, cudaStream_t stream);
+                              int n_steps, int epi, int sms, cudaStream_t stream);
 
 }  // namespace ra

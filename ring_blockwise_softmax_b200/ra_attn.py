@@ -43,7 +43,7 @@ SCHEDULES = {"stepwise": RA_RING_STEPWISE, "fused": RA_RING_FUSED}
 SYMBOLS = (
     "ra_attn_fwd", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_workspace_size",
     "ra_ring_fwd", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
-    "ra_status_string", "ra_last_error", "ra_version",
+    "ra_debug_exp2", "ra_status_string", "ra_last_error", "ra_version",
 )
 
 
@@ -71,6 +71,7 @@ _lib.ra_ring_fwd.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_in
 _lib.ra_get_device_status.argtypes = [_S]
 _lib.ra_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
 _lib.ra_debug_unarrived_wait.argtypes = [ctypes.c_uint64, _S]
+_lib.ra_debug_exp2.argtypes = [_F, _F, _F, ctypes.c_int64, _S]
 _lib.ra_status_string.argtypes = [ctypes.c_int]
 _lib.ra_status_string.restype = ctypes.c_char_p
 _lib.ra_last_error.argtypes = []
@@ -220,6 +221,11 @@ def set_wait_timeout_ns(ns: int):
 
 def debug_unarrived_wait(timeout_ns: int, stream=None):
     _check(_lib.ra_debug_unarrived_wait(int(timeout_ns), _stream(stream)), "ra_debug_unarrived_wait")
+
+
+def debug_exp2(x, y_poly=None, y_mufu=None, stream=None):
+    """ra_debug_exp2 on contiguous fp32 device tensors."""
+    _check(_lib.ra_debug_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), x.numel(), _stream(stream)), "ra_debug_exp2")
 
 
 # ---------------------------------------------------------------------------------------------

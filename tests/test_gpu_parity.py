@@ -279,3 +279,36 @@ def test_argument_errors_on_device(ra):
     with pytest.raises(ra.RaError) as e:
         ra.ring_fwd(q, k, v, 2, "contiguous", False, o, schedule="stepwise")  # no workspace
     assert e.value.status == ra.RA_ERR_WORKSPACE
+
+
+def test_exp2_routines_within_their_error_bounds(ra):
+    """The FMA-pipe exp2 polynomial stays within its derived 7.5e-5 relative bound (plus fp32
+    rounding) of 2^x over the range the softmax feeds it; the MUFU ex2 within 2^-21."""
+    xs = np.concatenate([np.linspace(-126.0, 8.0, 1_000_001), np.random.default_rng(0).uniform(-30, 0, 100_000)])
+    x = torch.tensor(xs, dtype=torch.float32, device="cuda")
+    yp = torch.empty_like(x)
+    ym = torch.empty_like(x)
+    ra.debug_exp2(x, yp, ym)
+    torch.cuda.synchronize()
+    xf = x.double().cpu().numpy()  # the exact fp32 inputs
+    ref = np.exp2(xf)
+    rel_p = np.abs(yp.double().cpu().numpy() - ref) / ref
+    rel_m = np.abs(ym.double().cpu().numpy() - ref) / ref
+    normal = xf > -125.0  # below that the result is subnormal / flushed
+    assert rel_p[normal].max() <= 7.6e-5, rel_p[normal].max()
+    assert rel_m[normal].max() <= 2.0 ** -21, rel_m[normal].max()
+    assert np.all(yp.cpu().numpy()[xf <= -126.0] < 2e-38)  # clamped inputs stay negligible
+
+
+@pytest.mark.parametrize("schedule", ["stepwise", "fused"])
+def test_ring_more_items_than_sms(ra, schedule):
+    """More 256-row work items than SMs, so each persistent CTA walks several items, including
+    runs of items whose keys are all in the causal future (contiguous shards s > r)."""
+    q, k, v = I.make_small(2, 16, 2048, 64, "bf16", seed=123)
+    qd, kd, vd = _dev(q, k, v)
+    o, lse = ra.ring_attention(qd, kd, vd, 8, "contiguous", True, schedule=schedule)
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == ra.RA_OK
+    rows = oracle.sample_rows(2048, 192, seed=5, must_include=[255, 256, 1791, 1792])
+    o_ref, l_ref = oracle_heads(to64(q), to64(k), to64(v), 1 / 8, True, rows=rows)
+    compare(to64(o)[:, :, rows], to64(lse)[:, :, rows], o_ref, l_ref, "bf16", f"many items {schedule}")
