@@ -11,21 +11,26 @@
 // "分布式注意力机制突破…" §3.4: align the maxima, rescale the sums).
 //
 // Structure (persistent: one CTA per SM walks work items; an item is 256 query rows = two
-// 128-row query tiles of one (batch, head, query shard); items are visited longest first):
+// 128-row query tiles of one (batch, head, query shard); items are numbered longest first and
+// dealt to the CTAs in a snake order):
 //   warps 0-3   softmax of query tile 0, thread i = row i = tensor-memory lane i
 //   warps 4-7   softmax of query tile 1
 //   warps 8-11  epilogue: normalise O, write O / LSE or LSE-merge into the accumulator
 //   warp 12     TMA producer: Q (two tiles) per item, then K_j / V_j into a STAGES-deep ring
-//   warp 13     MMA issuer (one thread): S_q = Q_q K_j^T (SS form), O_q += P_q V_j (TS form)
-// Both query tiles share every K/V tile (loaded once per 256 rows).  The MMA order per key
-// tile j is PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while one softmax warpgroup works on its
-// S, the tensor core runs the other tile's PV and next QK.
+//   warps 13,14 MMA issuers, one thread per query tile: S_q = Q_q K_j^T (SS form),
+//               O_q += P_q V_j (TS form)
+// Both query tiles share every K/V tile (loaded once per 256 rows).  Each query tile has its own
+// MMA-issuing thread, so while one softmax warpgroup works on its S the tensor core runs the
+// other tile's PV and next QK; with P in its own columns (DP <= 64) the next QK_q starts as soon
+// as S_q is in registers.
 // Tensor memory (512 columns): S_0, S_1 (128 fp32 columns each), O_0, O_1 (DP columns each),
 // and P_0, P_1 (bf16 pairs, 64 columns each) in their own columns when DP <= 64, otherwise over
 // the first half of S_q (then S_q is rewritten only after PV_q has consumed P_q).
-// Registers are rebalanced with setmaxnreg: softmax 168, epilogue 80, producer/MMA 96.
-// Part of the exponentials (1 in kEmuEvery columns of unmasked tiles) run as a polynomial on
-// the FMA pipe to offload the MUFU unit (exp2_poly3).
+// Registers are rebalanced with setmaxnreg (RegSplit): softmax 184, epilogue 64, producer/MMA 80
+// (176 / 80 / 80 for the merging epilogues).
+// Part of the exponentials (1 in kEmuEvery column pairs of unmasked tiles) can run as a
+// polynomial on the FMA pipe to offload the MUFU unit (exp2_poly3).  The softmax arithmetic
+// uses packed fp32x2 instructions and three-input max.
 // Every wait is bounded; on a timeout all roles stop, tensor memory is freed and the kernel
 // returns with the device status word set.
 #pragma once
@@ -55,28 +60,28 @@ struct FmhaCfg {
   static constexpr int P_COL0 = P_SEP ? 384 : 0;
   static constexpr int P_STRIDE = P_SEP ? 64 : 128;
   static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * STAGES);
-  static constexpr int NBAR = 3 + 3 * STAGES + 6 * 2;
+  static constexpr int NBAR = 3 + 3 * STAGES + 7 * 2;
   static constexpr int STATS_BYTES = 2 * 128 * 8;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES;
   static constexpr int THREADS = 512;
   static constexpr int D = DP;
 };
 
-#ifndef RA_REG_SOFTMAX
-#define RA_REG_SOFTMAX 168
-#endif
-#ifndef RA_REG_EPI
-#define RA_REG_EPI 80
-#endif
-#ifndef RA_REG_PROD
-#define RA_REG_PROD 96
-#endif
-static_assert(2 * 128 * RA_REG_SOFTMAX + 128 * RA_REG_EPI + 128 * RA_REG_PROD <= 65536, "register split too large");
+// Per-thread register budgets after setmaxnreg (softmax, epilogue, producer/MMA warpgroups).  The
+// merging epilogues (accumulate modes) need more registers than the plain output one.
+template <int EPI>
+struct RegSplit {
+  static constexpr bool kAcc = (EPI == 2 || EPI == 3);
+  static constexpr int kSoftmax = kAcc ? 176 : 184;
+  static constexpr int kEpi = kAcc ? 80 : 64;
+  static constexpr int kProd = 80;
+  static_assert(2 * 128 * kSoftmax + 128 * kEpi + 128 * kProd <= 65536, "register split exceeds the launch");
+};
 
 #ifndef RA_EMU_EVERY
 #define RA_EMU_EVERY 0
 #endif
-constexpr int kEmuEvery = RA_EMU_EVERY;  // 1 in kEmuEvery columns of unmasked tiles use the FMA-pipe exp2
+constexpr int kEmuEvery = RA_EMU_EVERY;  // 1 in kEmuEvery column pairs of unmasked tiles use the FMA-pipe exp2
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -99,6 +104,28 @@ __device__ __forceinline__ float exp2_poly3(float x) {
   p = fmaf(p, f, 0.9999280571937561f);
   // (bits(t) << 23) == n << 23 (mod 2^32): the constant part of bits(t) shifts out.
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two lanes of exp2_poly3 with packed fp32x2 arithmetic (same polynomial and range reduction).
+__device__ __forceinline__ float2 exp2_poly3_x2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, magic);
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));  // round(x), exact
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);                // x - round(x), exact
+  float2 p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                        make_float2(0.2426111251115799f, 0.2426111251115799f));
+  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -135,6 +162,14 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 // ---------------------------------------------------------------------------------------------
 // Work items and the walk over KV tiles
 // ---------------------------------------------------------------------------------------------
+// Items are numbered longest first; CTA c takes item c in round 0, G-1-c in round 1, G+c in
+// round 2, ... (a snake over the G persistent CTAs), which pairs long with short items.
+__device__ __forceinline__ int item_of_cta(int k) {
+  const int G = static_cast<int>(gridDim.x);
+  const int c = static_cast<int>(blockIdx.x);
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
+
 struct Item {
   int b, h, r, t0;
   int rows_valid[2];
@@ -200,6 +235,17 @@ __device__ __forceinline__ bool walk_next(Walk& k, const AttnWork& w, const Item
   return walk_seek(k, w, it, n_steps);
 }
 
+
+// Number of K/V tiles the item walks (what the MMA issuer needs; it never reads the keys).
+__device__ __forceinline__ int walk_count(const AttnWork& w, const Item& it, int n_steps) {
+  int n = 0;
+  for (int step = 0; step < n_steps; ++step) {
+    int s = (it.r - (w.ring_step + step)) % w.P;
+    if (s < 0) s += w.P;
+    n += (visible_key_limit(w, it.pos_last, s) + FmhaCfg<32>::BN - 1) / FmhaCfg<32>::BN;
+  }
+  return n;
+}
 
 // ---------------------------------------------------------------------------------------------
 // MMA issue (single thread) and the per-row epilogue
@@ -329,23 +375,29 @@ __device__ __forceinline__ void fmha_epilogue_row(const AttnWork& w, const Item&
 }
 
 // p = 2^(s * scale_log2 - base) for the 128 scores of this row, packed to bf16 pairs and stored
-// to tensor memory; partial row sums in rsp.  EMU: 1 in kEmuEvery columns on the FMA pipe (only
-// for tiles without masked scores, see exp2_poly3).
-template <bool EMU>
+// to tensor memory; row sums accumulated in two packed fp32x2 chains.  EVERY > 0: one column pair
+// in EVERY goes to the FMA-pipe polynomial instead of the MUFU (only for tiles without masked
+// scores, see exp2_poly3).
+template <int EVERY>
 __device__ __forceinline__ void softmax_exp_store(const uint32_t (&sr)[4][32], float sl2, float base, uint32_t p_addr,
-                                                  float (&rsp)[4]) {
+                                                  float2 (&rs)[2]) {
+  const float2 sc = make_float2(sl2, sl2);
+  const float2 nb = make_float2(-base, -base);
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float x0 = fmaf(__uint_as_float(sr[cc][2 * e]), sl2, -base);
-      const float x1 = fmaf(__uint_as_float(sr[cc][2 * e + 1]), sl2, -base);
-      const float p0 = ex2_approx(x0);
-      constexpr int kEvery = kEmuEvery > 0 ? kEmuEvery : 1;
-      const float p1 = (EMU && ((2 * e + 1) % kEvery) == kEvery - 1) ? exp2_poly3(x1) : ex2_approx(x1);
-      rsp[e & 3] += p0 + p1;
-      pk[e] = pack_bf16x2(p0, p1);
+      const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[cc][2 * e]), __uint_as_float(sr[cc][2 * e + 1])), sc, nb);
+      float2 p;
+      if (EVERY > 0 && (e % (EVERY > 0 ? EVERY : 1)) == (EVERY > 0 ? EVERY : 1) - 1) {
+        p = exp2_poly3_x2(x);
+      } else {
+        p.x = ex2_approx(x.x);
+        p.y = ex2_approx(x.y);
+      }
+      rs[e & 1] = __fadd2_rn(rs[e & 1], p);
+      pk[e] = pack_bf16x2(p.x, p.y);
     }
     tmem_st16(p_addr + cc * 16, pk);
   }
@@ -379,7 +431,8 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_o_full = bar_pv_done + 2;           // [2]
   uint64_t* bar_o_empty = bar_o_full + 2;           // [2]
   uint64_t* bar_stats = bar_o_empty + 2;            // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_stats + 2);
+  uint64_t* bar_s_free = bar_stats + 2;             // [2] softmax has loaded S_q into registers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s_free + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* stats = reinterpret_cast<float2*>(tmem_slot + 4);  // [2][128] (m_used, l_sum)
 
@@ -389,12 +442,12 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q_full, 1);
-    mbar_init(bar_q_empty, 1);
-    mbar_init(bar_mma_done, 1);
+    mbar_init(bar_q_empty, 2);   // one arrival per MMA issuer
+    mbar_init(bar_mma_done, 2);
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(bar_k_full + i, 1);
       mbar_init(bar_v_full + i, 1);
-      mbar_init(bar_kv_empty + i, 1);
+      mbar_init(bar_kv_empty + i, 2);  // one arrival per MMA issuer
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar_s_full + q, 1);
@@ -403,6 +456,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(bar_o_full + q, 1);
       mbar_init(bar_o_empty + q, 128);
       mbar_init(bar_stats + q, 128);
+      mbar_init(bar_s_free + q, 128);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -422,13 +476,15 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 12) {
-    setmaxnreg_dec<RA_REG_PROD>();
+    setmaxnreg_dec<RegSplit<EPI>::kProd>();
     if (warp == 12 && lane == 0) {
       // ================================================================ TMA producer
       int it_q = 0;
       long long g = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+      for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
+        const int idx = item_of_cta(k);
+        if (idx >= n_items) continue;
         Item it;
         decode_item(w, idx, it);
         Walk wk;
@@ -469,86 +525,83 @@ __global__ void __launch_bounds__(512, 1)
         mbar_drain(bar_k_full + j % C::STAGES, static_cast<uint32_t>(j / C::STAGES) & 1, w.wait_limit_ns);
         mbar_drain(bar_v_full + j % C::STAGES, static_cast<uint32_t>(j / C::STAGES) & 1, w.wait_limit_ns);
       }
-    } else if (warp == 13 && lane == 0) {
-      // ================================================================ MMA issuer
+    } else if ((warp == 13 || warp == 14) && lane == 0) {
+      // ================================================================ MMA issuers
+      // One thread per query tile q (warp 13: q = 0, warp 14: q = 1).  Each blocks on its own next
+      // event and issues, per key tile j:
+      //   QK_q(j+1) once K_{j+1} is loaded and S_q is free: with P in its own columns, as soon as
+      //             the softmax has loaded S_q(j) into registers (s_free); with P over S, once
+      //             PV_q(j) has completed (pv_done);
+      //   PV_q(j)   once P_q(j) is written (p_full), V_j is loaded and, for the first tile of an
+      //             item, the epilogue is done with O_q of the previous item (o_empty).
+      // A K/V stage is released when both issuers have committed it (kv_empty counts 2), and Q
+      // when both have issued their last QK of the item (q_empty counts 2).  The issuer that is
+      // behind never waits on the one ahead, so the two cannot deadlock.
+      const int q = warp - 13;
       constexpr uint32_t idesc_qk = make_idesc_bf16(128, C::BN, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, DP, 0, 1);
-      const uint32_t q_base = smem_addr(sQ);
+      const uint32_t q_addr = smem_addr(sQ) + q * C::TILE_BYTES;
       const uint32_t k_base = smem_addr(sK);
       const uint32_t v_base = smem_addr(sV);
+      const uint32_t d_s = tmem + C::S_COL0 + 128 * q;
+      const uint32_t d_o = tmem + C::O_COL0 + C::O_STRIDE * q;
+      const uint32_t p_t = tmem + C::P_COL0 + C::P_STRIDE * q;
       const DescBase<C> db;
       int it_all = 0, it_q = 0;
       long long g = 0;
-      int c[2] = {0, 0};  // PVs issued per query tile (all items)
+      int cq = 0;   // QKs issued for this query tile (all items)
+      int cpv = 0;  // PVs issued for this query tile (all items)
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+      auto qk = [&](long long gk, bool last_of_item) -> bool {
+        // S_q must be free: the previous QK's S consumed (own P columns) or its PV done (P over S).
+        if (cq > 0) {
+          if (C::P_SEP) {
+            if (!mbar_wait(bar_s_free + q, (cq - 1) & 1, ctl, 0x202)) return false;
+          } else {
+            if (!mbar_wait(bar_pv_done + q, (cq - 1) & 1, ctl, 0x203)) return false;
+          }
+        }
+        if (!mbar_wait(bar_k_full + gk % C::STAGES, static_cast<uint32_t>(gk / C::STAGES) & 1, ctl, 0x204))
+          return false;
+        tc_fence_after();
+        fmha_issue_qk<C>(db, d_s, q_addr, k_base + static_cast<int>(gk % C::STAGES) * C::TILE_BYTES, idesc_qk);
+        mma_commit(bar_s_full + q);
+        ++cq;
+        if (last_of_item) mma_commit(bar_q_empty);
+        return true;
+      };
+      for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
+        const int idx = item_of_cta(k);
+        if (idx >= n_items) continue;
         Item it;
         decode_item(w, idx, it);
-        Walk wk;
-        const bool has = walk_begin(wk, w, it, n_steps);
-        if (has) {
-          ok = mbar_wait(bar_q_full, it_q & 1, ctl, 0x201);
-          if (ok) ok = mbar_wait(bar_k_full + g % C::STAGES, static_cast<uint32_t>(g / C::STAGES) & 1, ctl, 0x202);
-          if (!ok) break;
-          tc_fence_after();
-          for (int q = 0; q < 2 && ok; ++q) {
-            // S_q may be rewritten once the previous PV_q has consumed P_q (aliased layout).
-            if (!C::P_SEP && c[q] > 0) ok = mbar_wait(bar_pv_done + q, (c[q] - 1) & 1, ctl, 0x203);
+        const int n = walk_count(w, it, n_steps);
+        if (n > 0) {
+          ok = mbar_wait(bar_q_full, it_q & 1, ctl, 0x201) && qk(g, n == 1);
+          for (int j = 0; ok && j < n; ++j) {
+            const long long gj = g + j;
+            if (C::P_SEP && j + 1 < n && !(ok = qk(gj + 1, j + 2 == n))) break;
+            ok = mbar_wait(bar_p_full + q, cpv & 1, ctl, 0x205) &&
+                 mbar_wait(bar_v_full + gj % C::STAGES, static_cast<uint32_t>(gj / C::STAGES) & 1, ctl, 0x206) &&
+                 (j > 0 || it_all == 0 || mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x207));
             if (!ok) break;
             tc_fence_after();
-            fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
-                             k_base + static_cast<int>(g % C::STAGES) * C::TILE_BYTES, idesc_qk);
-            mma_commit(bar_s_full + q);
+            fmha_issue_pv<C>(db, d_o, p_t, v_base + static_cast<int>(gj % C::STAGES) * C::TILE_BYTES, idesc_pv,
+                             j > 0);
+            mma_commit(bar_pv_done + q);
+            ++cpv;
+            mma_commit(bar_kv_empty + gj % C::STAGES);
+            if (!C::P_SEP && j + 1 < n && !(ok = qk(gj + 1, j + 2 == n))) break;
           }
           if (!ok) break;
-          int j = 0;
-          while (true) {
-            const long long gj = g + j;
-            const int st = static_cast<int>(gj % C::STAGES);
-            Walk nx = wk;
-            const bool has_next = walk_next(nx, w, it, n_steps);
-            if (!has_next) mma_commit(bar_q_empty);  // every QK of this item has been issued
-            for (int q = 0; q < 2 && ok; ++q) {
-              ok = mbar_wait(bar_p_full + q, c[q] & 1, ctl, 0x204);
-              if (ok && q == 0)
-                ok = mbar_wait(bar_v_full + st, static_cast<uint32_t>(gj / C::STAGES) & 1, ctl, 0x205);
-              if (ok && j == 0 && it_all > 0) ok = mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x206);
-              if (!ok) break;
-              tc_fence_after();
-              fmha_issue_pv<C>(db, tmem + C::O_COL0 + C::O_STRIDE * q, tmem + C::P_COL0 + C::P_STRIDE * q,
-                               v_base + st * C::TILE_BYTES, idesc_pv, j > 0);
-              mma_commit(bar_pv_done + q);
-              ++c[q];
-              if (has_next) {
-                const long long gn = gj + 1;
-                if (q == 0)
-                  ok = mbar_wait(bar_k_full + gn % C::STAGES, static_cast<uint32_t>(gn / C::STAGES) & 1, ctl, 0x207);
-                if (ok && !C::P_SEP) ok = mbar_wait(bar_pv_done + q, (c[q] - 1) & 1, ctl, 0x208);
-                if (!ok) break;
-                tc_fence_after();
-                fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
-                                 k_base + static_cast<int>(gn % C::STAGES) * C::TILE_BYTES, idesc_qk);
-                mma_commit(bar_s_full + q);
-              }
-            }
-            if (!ok) break;
-            mma_commit(bar_kv_empty + st);
-            ++j;
-            if (!has_next) break;
-            wk = nx;
-          }
-          if (!ok) break;
-          g += j;
+          mma_commit(bar_o_full + q);  // O_q of this item is final once these MMAs land
+          g += n;
           ++it_q;
+        } else {
+          // No PV in this item; still keep o_full at most one phase ahead of the epilogue.
+          if (it_all > 0 && !(ok = mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x208))) break;
+          mma_commit(bar_o_full + q);
         }
-        if (!has && it_all > 0) {
-          // An item with no visible key issues no PV; still keep o_full at most one phase ahead
-          // of the epilogue warps, which wait on it by parity.
-          for (int q = 0; q < 2 && ok; ++q) ok = mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x209);
-          if (!ok) break;
-        }
-        mma_commit(bar_o_full + 0);
-        mma_commit(bar_o_full + 1);
         ++it_all;
       }
       // Tensor memory is freed only after every MMA issued here has completed.
@@ -556,7 +609,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_drain(bar_mma_done, 0, w.wait_limit_ns);
     }
   } else if (warp < 8) {
-    setmaxnreg_inc<RA_REG_SOFTMAX>();
+    setmaxnreg_inc<RegSplit<EPI>::kSoftmax>();
     // ================================================================ softmax (query tile q)
     const int q = warp >> 2;
     const int row = threadIdx.x & 127;
@@ -567,7 +620,9 @@ __global__ void __launch_bounds__(512, 1)
     const float sl2 = w.scale_log2;
     int it_all = 0, c = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+    for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
+        const int idx = item_of_cta(k);
+        if (idx >= n_items) continue;
       Item it;
       decode_item(w, idx, it);
       const bool row_ok = row < it.rows_valid[q];
@@ -591,6 +646,11 @@ __global__ void __launch_bounds__(512, 1)
         reg_dep(sr[1]);
         reg_dep(sr[2]);
         reg_dep(sr[3]);
+        if (C::P_SEP) {
+          // S_q is in registers: the next QK_q may overwrite it while this tile's softmax runs.
+          tc_fence_before();
+          mbar_arrive(bar_s_free + q);
+        }
         const int lim = row_lim - wk.u0;  // keys [0, lim) of this tile are visible to this row
         const bool masked = __any_sync(0xffffffffu, lim < C::BN);
         if (lim < C::BN) {
@@ -604,9 +664,10 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) mxp[i] = __uint_as_float(sr[0][i]);
 #pragma unroll
-        for (int e = 8; e < 128; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], __uint_as_float(sr[e >> 5][e & 31]));
-        const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                               fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        for (int e = 8; e < 128; e += 2)
+          mxp[(e >> 1) & 7] = fmax3(mxp[(e >> 1) & 7], __uint_as_float(sr[e >> 5][e & 31]),
+                                    __uint_as_float(sr[(e + 1) >> 5][(e + 1) & 31]));
+        const float mx = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
         const float m_tile = mx * sl2;
         float m_new = m_used;
         float alpha = 1.f;
@@ -629,11 +690,11 @@ __global__ void __launch_bounds__(512, 1)
           if (!ok) break;
           tc_fence_after();
         }
-        float rsp[4] = {0.f, 0.f, 0.f, 0.f};  // row sum as 4 independent chains
+        float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // packed row sums
         if (masked || kEmuEvery == 0)
-          softmax_exp_store<false>(sr, sl2, base, p_addr, rsp);
+          softmax_exp_store<0>(sr, sl2, base, p_addr, rsp);
         else
-          softmax_exp_store<true>(sr, sl2, base, p_addr, rsp);
+          softmax_exp_store<kEmuEvery>(sr, sl2, base, p_addr, rsp);
         if (any_rescale) {
 #pragma unroll
           for (int cc = 0; cc < DP / 32; ++cc) {
@@ -641,11 +702,16 @@ __global__ void __launch_bounds__(512, 1)
             tmem_ld32(o_addr + cc * 32, orow);
             tmem_ld_wait(orow);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v = __fmul2_rn(make_float2(__uint_as_float(orow[e]), __uint_as_float(orow[e + 1])),
+                                          make_float2(alpha, alpha));
+              orow[e] = __float_as_uint(v.x);
+              orow[e + 1] = __float_as_uint(v.y);
+            }
             tmem_st32(o_addr + cc * 32, orow);
           }
         }
-        l_sum = l_sum * alpha + ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3]));
+        l_sum = l_sum * alpha + ((rsp[0].x + rsp[0].y) + (rsp[1].x + rsp[1].y));
         m_used = m_new;
         tmem_st_wait();
         tc_fence_before();
@@ -663,13 +729,15 @@ __global__ void __launch_bounds__(512, 1)
       ++it_all;
     }
   } else {
-    setmaxnreg_dec<RA_REG_EPI>();
+    setmaxnreg_dec<RegSplit<EPI>::kEpi>();
     // ================================================================ epilogue (both tiles)
     const int row = threadIdx.x & 127;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     int it_all = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+    for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
+        const int idx = item_of_cta(k);
+        if (idx >= n_items) continue;
       Item it;
       decode_item(w, idx, it);
       Walk wk;
