@@ -26,8 +26,8 @@
 // Tensor memory (512 columns): S_0, S_1 (128 fp32 columns each), O_0, O_1 (DP columns each),
 // and P_0, P_1 (bf16 pairs, 64 columns each) in their own columns when DP <= 64, otherwise over
 // the first half of S_q (then S_q is rewritten only after PV_q has consumed P_q).
-// Registers are rebalanced with setmaxnreg (RegSplit): softmax 184, epilogue 64, producer/MMA 80
-// (176 / 80 / 80 for the merging epilogues).
+// Registers are rebalanced with setmaxnreg (RegSplit): producer/MMA 80, epilogue 64 (80 when
+// merging), softmax the rest (176-184).
 // Part of the exponentials (1 in kEmuEvery column pairs of unmasked tiles) can run as a
 // polynomial on the FMA pipe to offload the MUFU unit (exp2_poly3).  The softmax arithmetic
 // uses packed fp32x2 instructions and three-input max.
@@ -54,6 +54,9 @@ struct FmhaCfg {
   static constexpr int TILE_BYTES = 128 * DP * 2;
   static constexpr int STAGES = (DP == 128) ? 2 : (DP == 64 ? 5 : 8);
   static constexpr bool P_SEP = DP <= 64;
+  // P in its own columns: one MMA issuer per query tile.  P over S: one issuer in a fixed
+  // PV_0, QK_0, PV_1, QK_1 order, which staggers the two tiles on the tensor core.
+  static constexpr int ISSUERS = P_SEP ? 2 : 1;
   static constexpr int S_COL0 = 0;
   static constexpr int O_COL0 = 256;
   static constexpr int O_STRIDE = (DP == 128) ? 128 : 64;
@@ -69,12 +72,12 @@ struct FmhaCfg {
 
 // Per-thread register budgets after setmaxnreg (softmax, epilogue, producer/MMA warpgroups).  The
 // merging epilogues (accumulate modes) need more registers than the plain output one.
-template <int EPI>
+template <int DP, int EPI>
 struct RegSplit {
   static constexpr bool kAcc = (EPI == 2 || EPI == 3);
-  static constexpr int kSoftmax = kAcc ? 176 : 184;
-  static constexpr int kEpi = kAcc ? 80 : 64;
   static constexpr int kProd = 80;
+  static constexpr int kEpi = kAcc ? 80 : 64;
+  static constexpr int kSoftmax = ((65536 / 128 - kProd - kEpi) / 2) / 8 * 8;
   static_assert(2 * 128 * kSoftmax + 128 * kEpi + 128 * kProd <= 65536, "register split exceeds the launch");
 };
 
@@ -147,6 +150,31 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > limit_ns) break;
+  }
+}
+
+#ifndef RA_ISSUER_SPIN
+#define RA_ISSUER_SPIN 1
+#endif
+// Wait used by the single-thread MMA issuers: spin on the non-blocking test (a sleeping try_wait
+// wakes up late, and each issuer hop sits on the critical path of a query tile), bounded like
+// mbar_wait.
+__device__ __forceinline__ bool mbar_wait_issuer(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, unsigned site) {
+  if (!RA_ISSUER_SPIN) return mbar_wait(bar, parity, ctl, site);
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
+    if (*ctl.abort) return false;
+    if (globaltimer_ns() - t0 > ctl.limit_ns) {
+      atomicOr(ctl.status, kDevStatusTimeout);
+      atomicCAS(ctl.status + 1, 0u, site);
+      *ctl.abort = 1;
+      __threadfence_block();
+      return false;
+    }
   }
 }
 
@@ -442,12 +470,12 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q_full, 1);
-    mbar_init(bar_q_empty, 2);   // one arrival per MMA issuer
-    mbar_init(bar_mma_done, 2);
+    mbar_init(bar_q_empty, C::ISSUERS);   // one arrival per MMA issuer
+    mbar_init(bar_mma_done, C::ISSUERS);
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(bar_k_full + i, 1);
       mbar_init(bar_v_full + i, 1);
-      mbar_init(bar_kv_empty + i, 2);  // one arrival per MMA issuer
+      mbar_init(bar_kv_empty + i, C::ISSUERS);  // one arrival per MMA issuer
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar_s_full + q, 1);
@@ -476,7 +504,7 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 12) {
-    setmaxnreg_dec<RegSplit<EPI>::kProd>();
+    setmaxnreg_dec<RegSplit<DP, EPI>::kProd>();
     if (warp == 12 && lane == 0) {
       // ================================================================ TMA producer
       int it_q = 0;
@@ -525,7 +553,88 @@ __global__ void __launch_bounds__(512, 1)
         mbar_drain(bar_k_full + j % C::STAGES, static_cast<uint32_t>(j / C::STAGES) & 1, w.wait_limit_ns);
         mbar_drain(bar_v_full + j % C::STAGES, static_cast<uint32_t>(j / C::STAGES) & 1, w.wait_limit_ns);
       }
-    } else if ((warp == 13 || warp == 14) && lane == 0) {
+    } else if (!C::P_SEP && warp == 13 && lane == 0) {
+      // ================================================================ MMA issuer (P over S)
+      // One thread, fixed order per key tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).  QK_q(j+1)
+      // rewrites S_q, which holds P_q(j), so it waits for PV_q(j) to complete; meanwhile the
+      // tensor core runs the other tile's work, and the two query tiles stay staggered.
+      constexpr uint32_t idesc_qk = make_idesc_bf16(128, C::BN, 0, 0);
+      constexpr uint32_t idesc_pv = make_idesc_bf16(128, DP, 0, 1);
+      const uint32_t q_base = smem_addr(sQ);
+      const uint32_t k_base = smem_addr(sK);
+      const uint32_t v_base = smem_addr(sV);
+      const DescBase<C> db;
+      int it_all = 0, it_q = 0;
+      long long g = 0;
+      // Every query tile processes every K/V tile, so the per-tile barrier phases all follow the
+      // CTA's running K/V tile index g + j.
+      bool ok = true;
+      for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
+        const int idx = item_of_cta(k);
+        if (idx >= n_items) continue;
+        Item it;
+        decode_item(w, idx, it);
+        const int n = walk_count(w, it, n_steps);
+        if (n == 0) {
+          for (int q = 0; q < 2 && ok && it_all > 0; ++q)
+            ok = mbar_wait_issuer(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x208);
+          if (!ok) break;
+          mma_commit(bar_o_full + 0);
+          mma_commit(bar_o_full + 1);
+          ++it_all;
+          continue;
+        }
+        ok = mbar_wait_issuer(bar_q_full, it_q & 1, ctl, 0x201) &&
+             mbar_wait_issuer(bar_k_full + g % C::STAGES, static_cast<uint32_t>(g / C::STAGES) & 1, ctl, 0x204);
+        for (int q = 0; q < 2 && ok; ++q) {
+          if (g > 0 && !(ok = mbar_wait_issuer(bar_pv_done + q, static_cast<uint32_t>(g - 1) & 1, ctl, 0x203))) break;
+          tc_fence_after();
+          fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
+                           k_base + static_cast<int>(g % C::STAGES) * C::TILE_BYTES, idesc_qk);
+          mma_commit(bar_s_full + q);
+        }
+        if (!ok) break;
+        if (n == 1) mma_commit(bar_q_empty);
+        for (int j = 0; ok && j < n; ++j) {
+          const long long gj = g + j;
+          const bool has_next = j + 1 < n;
+          for (int q = 0; q < 2 && ok; ++q) {
+            ok = mbar_wait_issuer(bar_p_full + q, static_cast<uint32_t>(gj) & 1, ctl, 0x205) &&
+                 (q == 1 || mbar_wait_issuer(bar_v_full + gj % C::STAGES, static_cast<uint32_t>(gj / C::STAGES) & 1, ctl,
+                                             0x206)) &&
+                 (j > 0 || it_all == 0 || mbar_wait_issuer(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x207));
+            if (!ok) break;
+            tc_fence_after();
+            fmha_issue_pv<C>(db, tmem + C::O_COL0 + C::O_STRIDE * q, tmem + C::P_COL0 + C::P_STRIDE * q,
+                             v_base + static_cast<int>(gj % C::STAGES) * C::TILE_BYTES, idesc_pv, j > 0);
+            mma_commit(bar_pv_done + q);
+            if (has_next) {
+              const long long gn = gj + 1;
+              ok = (q == 1 || mbar_wait_issuer(bar_k_full + gn % C::STAGES, static_cast<uint32_t>(gn / C::STAGES) & 1,
+                                               ctl, 0x209)) &&
+                   mbar_wait_issuer(bar_pv_done + q, static_cast<uint32_t>(gj) & 1, ctl, 0x20a);
+              if (!ok) break;
+              tc_fence_after();
+              fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
+                               k_base + static_cast<int>(gn % C::STAGES) * C::TILE_BYTES, idesc_qk);
+              mma_commit(bar_s_full + q);
+              if (q == 1 && j + 2 == n) mma_commit(bar_q_empty);  // last QKs of the item issued
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar_kv_empty + gj % C::STAGES);
+        }
+        if (!ok) break;
+        mma_commit(bar_o_full + 0);
+        mma_commit(bar_o_full + 1);
+        g += n;
+        ++it_q;
+        ++it_all;
+      }
+      // Tensor memory is freed only after every MMA issued here has completed.
+      mma_commit(bar_mma_done);
+      mbar_drain(bar_mma_done, 0, w.wait_limit_ns);
+    } else if (C::P_SEP && (warp == 13 || warp == 14) && lane == 0) {
       // ================================================================ MMA issuers
       // One thread per query tile q (warp 13: q = 0, warp 14: q = 1).  Each blocks on its own next
       // event and issues, per key tile j:
@@ -556,12 +665,12 @@ __global__ void __launch_bounds__(512, 1)
         // S_q must be free: the previous QK's S consumed (own P columns) or its PV done (P over S).
         if (cq > 0) {
           if (C::P_SEP) {
-            if (!mbar_wait(bar_s_free + q, (cq - 1) & 1, ctl, 0x202)) return false;
+            if (!mbar_wait_issuer(bar_s_free + q, (cq - 1) & 1, ctl, 0x202)) return false;
           } else {
-            if (!mbar_wait(bar_pv_done + q, (cq - 1) & 1, ctl, 0x203)) return false;
+            if (!mbar_wait_issuer(bar_pv_done + q, (cq - 1) & 1, ctl, 0x203)) return false;
           }
         }
-        if (!mbar_wait(bar_k_full + gk % C::STAGES, static_cast<uint32_t>(gk / C::STAGES) & 1, ctl, 0x204))
+        if (!mbar_wait_issuer(bar_k_full + gk % C::STAGES, static_cast<uint32_t>(gk / C::STAGES) & 1, ctl, 0x204))
           return false;
         tc_fence_after();
         fmha_issue_qk<C>(db, d_s, q_addr, k_base + static_cast<int>(gk % C::STAGES) * C::TILE_BYTES, idesc_qk);
@@ -577,13 +686,13 @@ __global__ void __launch_bounds__(512, 1)
         decode_item(w, idx, it);
         const int n = walk_count(w, it, n_steps);
         if (n > 0) {
-          ok = mbar_wait(bar_q_full, it_q & 1, ctl, 0x201) && qk(g, n == 1);
+          ok = mbar_wait_issuer(bar_q_full, it_q & 1, ctl, 0x201) && qk(g, n == 1);
           for (int j = 0; ok && j < n; ++j) {
             const long long gj = g + j;
             if (C::P_SEP && j + 1 < n && !(ok = qk(gj + 1, j + 2 == n))) break;
-            ok = mbar_wait(bar_p_full + q, cpv & 1, ctl, 0x205) &&
-                 mbar_wait(bar_v_full + gj % C::STAGES, static_cast<uint32_t>(gj / C::STAGES) & 1, ctl, 0x206) &&
-                 (j > 0 || it_all == 0 || mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x207));
+            ok = mbar_wait_issuer(bar_p_full + q, cpv & 1, ctl, 0x205) &&
+                 mbar_wait_issuer(bar_v_full + gj % C::STAGES, static_cast<uint32_t>(gj / C::STAGES) & 1, ctl, 0x206) &&
+                 (j > 0 || it_all == 0 || mbar_wait_issuer(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x207));
             if (!ok) break;
             tc_fence_after();
             fmha_issue_pv<C>(db, d_o, p_t, v_base + static_cast<int>(gj % C::STAGES) * C::TILE_BYTES, idesc_pv,
@@ -599,7 +708,7 @@ __global__ void __launch_bounds__(512, 1)
           ++it_q;
         } else {
           // No PV in this item; still keep o_full at most one phase ahead of the epilogue.
-          if (it_all > 0 && !(ok = mbar_wait(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x208))) break;
+          if (it_all > 0 && !(ok = mbar_wait_issuer(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x208))) break;
           mma_commit(bar_o_full + q);
         }
         ++it_all;
@@ -609,7 +718,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_drain(bar_mma_done, 0, w.wait_limit_ns);
     }
   } else if (warp < 8) {
-    setmaxnreg_inc<RegSplit<EPI>::kSoftmax>();
+    setmaxnreg_inc<RegSplit<DP, EPI>::kSoftmax>();
     // ================================================================ softmax (query tile q)
     const int q = warp >> 2;
     const int row = threadIdx.x & 127;
@@ -729,7 +838,7 @@ __global__ void __launch_bounds__(512, 1)
       ++it_all;
     }
   } else {
-    setmaxnreg_dec<RegSplit<EPI>::kEpi>();
+    setmaxnreg_dec<RegSplit<DP, EPI>::kEpi>();
     // ================================================================ epilogue (both tiles)
     const int row = threadIdx.x & 127;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
