@@ -161,6 +161,26 @@ ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
                         const ra_tensor_t* o, float* lse, const ra_stream_t* streams,
                         int n_streams, void* workspace, size_t workspace_bytes);
 
+/* ra_ring_fwd with the RA_RING_STEPWISE schedule for callers that cannot allocate device memory
+ * at the point of the call: code recording a CUDA graph (cudaMalloc cannot be captured), code
+ * whose device memory is entirely held by another allocator, or latency-critical paths that
+ * must not pay for an allocation's implicit synchronisation.  There is no counterpart on the
+ * source pages: this is an interface convenience of this library.
+ * The fp32 (O, LSE) accumulator lives in a fixed array of RA_NOALLOC_SCRATCH_BYTES inside the
+ * library (held on every device that loads the library, until the process exits); nothing is
+ * allocated.  Problems whose accumulator (ra_ring_workspace_size with RA_RING_STEPWISE) exceeds
+ * that size are rejected with RA_ERR_WORKSPACE and a message naming both sizes.
+ * The first call on each device looks up the array's device address with that device current;
+ * make that first call before any stream capture.  All calls on a device share the one array:
+ * calls whose work overlaps on the GPU (different streams, or interleaved with ra_ring_fwd_noalloc
+ * calls on other threads) race on it, so order them on one stream.  The array keeps the last
+ * call's contents; no clearing is needed because ring step 0 overwrites every element the later
+ * steps read.  Other arguments and errors as for ra_ring_fwd (one stream). */
+#define RA_NOALLOC_SCRATCH_BYTES (32u << 20)
+ra_status_t ra_ring_fwd_noalloc(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P,
+                                int layout, int causal, float scale, const ra_tensor_t* o, float* lse,
+                                ra_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device status word that kernels set when a
  * bounded wait runs out (each wait gives up after ra_set_wait_timeout_ns(); the kernel then
  * stops its work, frees its tensor memory and returns, leaving its outputs undefined).

@@ -32,6 +32,7 @@ FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxa
 
 UNITS = [
     ("ra_attn.cu", "ra_attn.o", []),
+    ("ra_noalloc.cu", "ra_noalloc.o", []),
     ("ra_fmha_launch.cu", "fmha_dp32.o", ["-DRA_FMHA_DP=32"]),
     ("ra_fmha_launch.cu", "fmha_dp64.o", ["-DRA_FMHA_DP=64"]),
     ("ra_fmha_launch.cu", "fmha_dp128.o", ["-DRA_FMHA_DP=128"]),

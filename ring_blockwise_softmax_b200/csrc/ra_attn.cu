@@ -334,6 +334,11 @@ int q_rows_per_cta(int dtype) { return dtype == RA_BF16 ? 128 : ra::kSimtRows; }
 
 }  // namespace
 
+namespace ra {
+// Lets the library's other translation units report through ra_last_error().
+ra_status_t set_last_error(ra_status_t status, const char* message) { return fail(status, "%s", message); }
+}  // namespace ra
+
 // ==============================================================================================
 // Entry points
 // ==============================================================================================

@@ -42,7 +42,7 @@ SCHEDULES = {"stepwise": RA_RING_STEPWISE, "fused": RA_RING_FUSED}
 # Exported symbols of the library, in header order (the CPU test checks each one is present).
 SYMBOLS = (
     "ra_attn_fwd", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_workspace_size",
-    "ra_ring_fwd", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
+    "ra_ring_fwd", "ra_ring_fwd_noalloc", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
     "ra_debug_exp2", "ra_status_string", "ra_last_error", "ra_version",
 )
 
@@ -68,6 +68,8 @@ _lib.ra_lse_merge_n.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(
 _lib.ra_ring_workspace_size.argtypes = [_T, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
 _lib.ra_ring_fwd.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int, _T,
                              _F, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t]
+_lib.ra_ring_fwd_noalloc.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, _T, _F,
+                                     _S]
 _lib.ra_get_device_status.argtypes = [_S]
 _lib.ra_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
 _lib.ra_debug_unarrived_wait.argtypes = [ctypes.c_uint64, _S]
@@ -208,6 +210,17 @@ def ring_fwd(q, k, v, P: int, layout: str, causal: bool, o, lse=None, scale: flo
     _check(_lib.ra_ring_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), int(P), LAYOUTS[layout],
                             int(bool(causal)), float(scale), SCHEDULES[schedule], ctypes.byref(to), _ptr(lse), arr,
                             len(streams), ws_ptr, ws_bytes), "ra_ring_fwd")
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def ring_fwd_noalloc(q, k, v, P: int, layout: str, causal: bool, o, lse=None, scale: float = 0.0, stream=None):
+    """ra_ring_fwd_noalloc: the stepwise ring with the library's fixed scratch (no workspace)."""
+    tq, tk, tv, to = (tensor_desc(x) for x in (q, k, v, o))
+    _check(_lib.ra_ring_fwd_noalloc(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), int(P), LAYOUTS[layout],
+                                    int(bool(causal)), float(scale), ctypes.byref(to), _ptr(lse), _stream(stream)),
+           "ra_ring_fwd_noalloc")
 
 
 def get_device_status(stream=None) -> int:
