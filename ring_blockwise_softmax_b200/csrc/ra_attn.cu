@@ -334,6 +334,36 @@ int q_rows_per_cta(int dtype) { return dtype == RA_BF16 ? 128 : ra::kSimtRows; }
 
 }  // namespace
 
+namespace {
+// Launchers for the runtime lane-group size G (a power of two <= 32).
+template <int VEC>
+static void launch_merge2(int G, dim3 grid, cudaStream_t st, const float* o_a, const float* lse_a, const float* o_b,
+                          const float* lse_b, float* o_out, float* lse_out, long long rows, int d) {
+  switch (G) {
+    case 1: ra::lse_merge2_kernel<VEC, 1><<<grid, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d); break;
+    case 2: ra::lse_merge2_kernel<VEC, 2><<<grid, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d); break;
+    case 4: ra::lse_merge2_kernel<VEC, 4><<<grid, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d); break;
+    case 8: ra::lse_merge2_kernel<VEC, 8><<<grid, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d); break;
+    case 16: ra::lse_merge2_kernel<VEC, 16><<<grid, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d); break;
+    default: ra::lse_merge2_kernel<VEC, 32><<<grid, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d); break;
+  }
+}
+
+template <int VEC, int KMAX>
+static void launch_merge_n(int G, dim3 grid, cudaStream_t st, const ra::MergeParts& parts, int k, float* o_out,
+                           float* lse_out, long long rows, int d) {
+  switch (G) {
+    case 1: ra::lse_merge_n_kernel<VEC, 1, KMAX><<<grid, 256, 0, st>>>(parts, k, o_out, lse_out, rows, d); break;
+    case 2: ra::lse_merge_n_kernel<VEC, 2, KMAX><<<grid, 256, 0, st>>>(parts, k, o_out, lse_out, rows, d); break;
+    case 4: ra::lse_merge_n_kernel<VEC, 4, KMAX><<<grid, 256, 0, st>>>(parts, k, o_out, lse_out, rows, d); break;
+    case 8: ra::lse_merge_n_kernel<VEC, 8, KMAX><<<grid, 256, 0, st>>>(parts, k, o_out, lse_out, rows, d); break;
+    case 16: ra::lse_merge_n_kernel<VEC, 16, KMAX><<<grid, 256, 0, st>>>(parts, k, o_out, lse_out, rows, d); break;
+    default: ra::lse_merge_n_kernel<VEC, 32, KMAX><<<grid, 256, 0, st>>>(parts, k, o_out, lse_out, rows, d); break;
+  }
+}
+
+}  // namespace
+
 namespace ra {
 // Lets the library's other translation units report through ra_last_error().
 ra_status_t set_last_error(ra_status_t status, const char* message) { return fail(status, "%s", message); }
@@ -436,16 +466,6 @@ static int merge_group(int nv) {
   return g;
 }
 
-#define RA_MERGE_DISPATCH(KERNEL, VEC, G, ...)                                          \
-  switch (G) {                                                                          \
-    case 1: ra::KERNEL<VEC, 1><<<grid, 256, 0, st>>>(__VA_ARGS__); break;               \
-    case 2: ra::KERNEL<VEC, 2><<<grid, 256, 0, st>>>(__VA_ARGS__); break;               \
-    case 4: ra::KERNEL<VEC, 4><<<grid, 256, 0, st>>>(__VA_ARGS__); break;               \
-    case 8: ra::KERNEL<VEC, 8><<<grid, 256, 0, st>>>(__VA_ARGS__); break;               \
-    case 16: ra::KERNEL<VEC, 16><<<grid, 256, 0, st>>>(__VA_ARGS__); break;             \
-    default: ra::KERNEL<VEC, 32><<<grid, 256, 0, st>>>(__VA_ARGS__); break;             \
-  }
-
 static unsigned merge_grid(long long rows, int G, int sms) {
   const long long groups_per_block = 256 / G;
   long long blocks = (rows + groups_per_block - 1) / groups_per_block;
@@ -467,15 +487,12 @@ ra_status_t ra_lse_merge(const float* o_a, const float* lse_a, const float* o_b,
   if (s0 != RA_OK) return s0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool vec = d % 4 == 0 && aligned16(o_a) && aligned16(o_b) && aligned16(o_out);
-  if (vec) {
-    const int G = merge_group(d / 4);
-    dim3 grid(merge_grid(rows, G, dev.sms));
-    RA_MERGE_DISPATCH(lse_merge2_kernel, 4, G, o_a, lse_a, o_b, lse_b, o_out, lse_out, (long long)rows, d)
-  } else {
-    const int G = merge_group(d);
-    dim3 grid(merge_grid(rows, G, dev.sms));
-    RA_MERGE_DISPATCH(lse_merge2_kernel, 1, G, o_a, lse_a, o_b, lse_b, o_out, lse_out, (long long)rows, d)
-  }
+  const int G = merge_group(vec ? d / 4 : d);
+  dim3 grid(merge_grid(rows, G, dev.sms));
+  if (vec)
+    launch_merge2<4>(G, grid, st, o_a, lse_a, o_b, lse_b, o_out, lse_out, (long long)rows, d);
+  else
+    launch_merge2<1>(G, grid, st, o_a, lse_a, o_b, lse_b, o_out, lse_out, (long long)rows, d);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
   return ok();
@@ -500,14 +517,22 @@ ra_status_t ra_lse_merge_n(const float* const* o_parts, const float* const* lse_
   ra_status_t s0 = current_device(&dev);
   if (s0 != RA_OK) return s0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int G = merge_group(vec ? d / 4 : d);
+  dim3 grid(merge_grid(rows, G, dev.sms));
   if (vec) {
-    const int G = merge_group(d / 4);
-    dim3 grid(merge_grid(rows, G, dev.sms));
-    RA_MERGE_DISPATCH(lse_merge_n_kernel, 4, G, parts, k, o_out, lse_out, (long long)rows, d)
+    if (k <= 4)
+      launch_merge_n<4, 4>(G, grid, st, parts, k, o_out, lse_out, (long long)rows, d);
+    else if (k <= 8)
+      launch_merge_n<4, 8>(G, grid, st, parts, k, o_out, lse_out, (long long)rows, d);
+    else if (k <= 16)
+      launch_merge_n<4, 16>(G, grid, st, parts, k, o_out, lse_out, (long long)rows, d);
+    else
+      launch_merge_n<4, 32>(G, grid, st, parts, k, o_out, lse_out, (long long)rows, d);
   } else {
-    const int G = merge_group(d);
-    dim3 grid(merge_grid(rows, G, dev.sms));
-    RA_MERGE_DISPATCH(lse_merge_n_kernel, 1, G, parts, k, o_out, lse_out, (long long)rows, d)
+    if (k <= 8)
+      launch_merge_n<1, 8>(G, grid, st, parts, k, o_out, lse_out, (long long)rows, d);
+    else
+      launch_merge_n<1, 32>(G, grid, st, parts, k, o_out, lse_out, (long long)rows, d);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) lse_merge2_kernel(const float* o_a, const
       const V* pa = reinterpret_cast<const V*>(o_a + row * d);
       const V* pb = reinterpret_cast<const V*>(o_b + row * d);
       V* po = reinterpret_cast<V*>(o_out + row * d);
-      for (int c = g; c < nv; c += G) po[c] = axpby(wa, pa[c], wb, pb[c]);
+      for (int c = g; c < nv; c += G) __stcs(po + c, axpby(wa, __ldcs(pa + c), wb, __ldcs(pb + c)));
     }
     __syncwarp();
     if (active && g == 0) lse_out[row] = L;
@@ -74,7 +74,9 @@ struct MergeParts {
   const float* l[32];
 };
 
-template <int VEC, int G>
+// KMAX >= k: the part loops are unrolled KMAX times and predicated on i < k, so the weights stay
+// in registers and the k loads of one vector are issued back to back.
+template <int VEC, int G, int KMAX>
 __global__ void __launch_bounds__(256) lse_merge_n_kernel(const MergeParts parts, int k, float* o_out,
                                                           float* lse_out, long long rows, int d) {
   using V = typename VecT<VEC>::T;
@@ -90,28 +92,29 @@ __global__ void __launch_bounds__(256) lse_merge_n_kernel(const MergeParts parts
     const bool active = row < rows;
     float L = -INFINITY;
     if (active) {
-      float wgt[32];
+      float wgt[KMAX];
       float m = -INFINITY;
-      for (int i = 0; i < k; ++i) {
-        wgt[i] = parts.l[i][row];
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i) {
+        wgt[i] = (i < k) ? parts.l[i][row] : -INFINITY;
         m = fmaxf(m, wgt[i]);
       }
       float ssum = 0.f;
-      if (m != -INFINITY) {
-        for (int i = 0; i < k; ++i) {
-          wgt[i] = expf(wgt[i] - m);  // e^{-inf} = 0 for empty partials
-          ssum += wgt[i];
-        }
-        L = m + logf(ssum);
-      } else {
-        for (int i = 0; i < k; ++i) wgt[i] = 0.f;
+      const float m_safe = (m == -INFINITY) ? 0.f : m;
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i) {
+        wgt[i] = expf(wgt[i] - m_safe);  // e^{-inf} = 0 for empty partials and unused slots
+        ssum += wgt[i];
       }
+      if (m != -INFINITY) L = m + logf(ssum);
       const float inv = ssum > 0.f ? 1.f / ssum : 0.f;
       V* po = reinterpret_cast<V*>(o_out + row * d);
       for (int c = g; c < nv; c += G) {
         V acc = zero_v(static_cast<V*>(nullptr));
-        for (int i = 0; i < k; ++i) acc = fma4(wgt[i], reinterpret_cast<const V*>(parts.o[i] + row * d)[c], acc);
-        po[c] = scale_v(acc, inv);
+#pragma unroll
+        for (int i = 0; i < KMAX; ++i)
+          if (i < k) acc = fma4(wgt[i], __ldcs(reinterpret_cast<const V*>(parts.o[i] + row * d) + c), acc);
+        __stcs(po + c, scale_v(acc, inv));
       }
     }
     __syncwarp();
