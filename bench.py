@@ -33,6 +33,34 @@ SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def kernel_sources_hash() -> str:
+    """sha256 over the CUDA sources of the library (identifies the kernel build a capture is of)."""
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "ring_blockwise_softmax_b200", "csrc", "*.cu*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str, schedule: str):
+    """DRAM bytes per launch of the attention kernel from profiles/fmha_traffic.json, if that
+    capture was taken of the current kernel sources on this workload and schedule; else None."""
+    p = os.path.join(ROOT, "profiles", "fmha_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("kernel_sources_sha256") != kernel_sources_hash():
+        return None
+    for e in rec.get("captures", []):
+        if e.get("workload") == workload and e.get("schedule") == schedule:
+            return e.get("dram_bytes_per_launch")
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -365,7 +393,8 @@ def run_gpu(args, w):
         "pct_of_measured_bf16_peak": 100.0 * (value / world) / peak,
         "roofline": {"bound": "tensor", "kernel": "fmha_fwd_sm100", "achieved": value / world, "peak": peak,
                      "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s", "frac": (value / world) / peak,
-                     "traffic": args.traffic,
+                     "traffic": args.traffic if args.traffic is not None else recorded_traffic(f"cfg{w.cfg}",
+                                                                                                  args.schedule),
                      "note": "algorithmic FLOPs (4*B*H*N^2*d, halved when causal) / summed duration of the step's "
                              f"{launches_per_step} serialised launches (CUDA events on the launch stream)"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

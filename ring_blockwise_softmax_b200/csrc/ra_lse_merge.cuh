@@ -46,26 +46,54 @@ __global__ void __launch_bounds__(256) lse_merge2_kernel(const float* o_a, const
                                                          const float* o_b, const float* lse_b,
                                                          float* o_out, float* lse_out, long long rows, int d) {
   using V = typename VecT<VEC>::T;
+  constexpr int R = 2;  // rows per group and iteration: 2 x 2 loads in flight per lane
   const int nv = d / VEC;
   const int lane = threadIdx.x & 31;
   const int g = lane % G;
   const long long groups_per_block = blockDim.x / G;
   const long long first = static_cast<long long>(blockIdx.x) * groups_per_block + threadIdx.x / G;
   const long long stride = static_cast<long long>(gridDim.x) * groups_per_block;
-  const long long n_iter = (rows + stride - 1) / stride;  // same trip count for every lane of a warp
+  const long long n_iter = (rows + R * stride - 1) / (R * stride);  // same trip count in a warp
   for (long long it = 0; it < n_iter; ++it) {
-    const long long row = first + it * stride;
-    const bool active = row < rows;
-    float L = 0.f, wa = 0.f, wb = 0.f;
-    if (active) {
-      lse_merge_weights(lse_a[row], lse_b[row], L, wa, wb);
-      const V* pa = reinterpret_cast<const V*>(o_a + row * d);
-      const V* pb = reinterpret_cast<const V*>(o_b + row * d);
-      V* po = reinterpret_cast<V*>(o_out + row * d);
-      for (int c = g; c < nv; c += G) __stcs(po + c, axpby(wa, __ldcs(pa + c), wb, __ldcs(pb + c)));
+    long long row[R];
+    bool active[R];
+    V va[R], vb[R];
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr) {
+      row[rr] = first + (it * R + rr) * stride;
+      active[rr] = row[rr] < rows;
+      // The first column group's O loads go out before the LSE arithmetic (latencies overlap).
+      if (active[rr] && g < nv) {
+        va[rr] = __ldcs(reinterpret_cast<const V*>(o_a + row[rr] * d) + g);
+        vb[rr] = __ldcs(reinterpret_cast<const V*>(o_b + row[rr] * d) + g);
+      }
+    }
+    float L[R], wa[R], wb[R];
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr) {
+      L[rr] = 0.f;
+      wa[rr] = 0.f;
+      wb[rr] = 0.f;
+      if (active[rr]) lse_merge_weights(lse_a[row[rr]], lse_b[row[rr]], L[rr], wa[rr], wb[rr]);
+    }
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr) {
+      if (!active[rr]) continue;
+      const V* pa = reinterpret_cast<const V*>(o_a + row[rr] * d);
+      const V* pb = reinterpret_cast<const V*>(o_b + row[rr] * d);
+      V* po = reinterpret_cast<V*>(o_out + row[rr] * d);
+      for (int c = g; c < nv; c += G) {
+        if (c != g) {
+          va[rr] = __ldcs(pa + c);
+          vb[rr] = __ldcs(pb + c);
+        }
+        __stcs(po + c, axpby(wa[rr], va[rr], wb[rr], vb[rr]));
+      }
     }
     __syncwarp();
-    if (active && g == 0) lse_out[row] = L;
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr)
+      if (active[rr] && g == 0) lse_out[row[rr]] = L[rr];
   }
 }
 
@@ -92,6 +120,13 @@ __global__ void __launch_bounds__(256) lse_merge_n_kernel(const MergeParts parts
     const bool active = row < rows;
     float L = -INFINITY;
     if (active) {
+      // Issue this row's O loads for the first column group before the LSE arithmetic, so the
+      // two memory latencies overlap instead of adding up.
+      V ov[KMAX];
+      const bool first_ok = g < nv;
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i)
+        if (i < k && first_ok) ov[i] = __ldcs(reinterpret_cast<const V*>(parts.o[i] + row * d) + g);
       float wgt[KMAX];
       float m = -INFINITY;
 #pragma unroll
@@ -110,10 +145,15 @@ __global__ void __launch_bounds__(256) lse_merge_n_kernel(const MergeParts parts
       const float inv = ssum > 0.f ? 1.f / ssum : 0.f;
       V* po = reinterpret_cast<V*>(o_out + row * d);
       for (int c = g; c < nv; c += G) {
+        if (c != g) {
+#pragma unroll
+          for (int i = 0; i < KMAX; ++i)
+            if (i < k) ov[i] = __ldcs(reinterpret_cast<const V*>(parts.o[i] + row * d) + c);
+        }
         V acc = zero_v(static_cast<V*>(nullptr));
 #pragma unroll
         for (int i = 0; i < KMAX; ++i)
-          if (i < k) acc = fma4(wgt[i], __ldcs(reinterpret_cast<const V*>(parts.o[i] + row * d) + c), acc);
+          if (i < k) acc = fma4(wgt[i], ov[i], acc);
         __stcs(po + c, scale_v(acc, inv));
       }
     }
