@@ -33,15 +33,17 @@ SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+FMHA_SOURCES = ("ra_common.cuh", "ra_fmha_sm100.cuh", "ra_fmha_launch.cu")
+
+
 def kernel_sources_hash() -> str:
-    """sha256 over the CUDA sources of the library (identifies the kernel build a capture is of)."""
-    import glob
+    """sha256 over the attention kernel's sources (identifies the kernel build a capture is of)."""
     import hashlib
 
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "ring_blockwise_softmax_b200", "csrc", "*.cu*"))):
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    for name in FMHA_SOURCES:
+        with open(os.path.join(ROOT, "ring_blockwise_softmax_b200", "csrc", name), "rb") as fh:
+            h.update(name.encode() + b"\0" + fh.read())
     return h.hexdigest()
 
 

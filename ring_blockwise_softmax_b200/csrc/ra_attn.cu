@@ -232,9 +232,25 @@ struct Maps {
   CUtensorMap q, k, v;
 };
 
-ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::AttnWork& w, int n_steps, int epi,
+// Heads per work-item group: the largest divisor of B*H (equal groups keep the longest-first
+// balance inside each group) whose K and V, all shards, fit in ~80 MiB of the 126 MB L2.
+int heads_per_group(const ra::AttnWork& w, int elem_bytes) {
+  const double kv_bytes = 2.0 * static_cast<double>(w.n_kv) * w.P * w.d * elem_bytes;
+  const double budget = 80.0 * 1024 * 1024;
+  const long long bh = static_cast<long long>(w.B) * w.H;
+  long long hg_max = static_cast<long long>(budget / (kv_bytes > 1.0 ? kv_bytes : 1.0));
+  if (hg_max < 1) hg_max = 1;
+  if (hg_max >= bh) return static_cast<int>(bh);
+  for (long long hg = hg_max; hg > 1; --hg)
+    if (bh % hg == 0) return static_cast<int>(hg);
+  return 1;
+}
+
+ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::AttnWork& w_in, int n_steps, int epi,
                              int sms, cudaStream_t stream) {
-  if (w.B > 65535 || w.H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
+  if (w_in.B > 65535 || w_in.H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
+  ra::AttnWork w = w_in;
+  w.hgroup = heads_per_group(w, q->dtype == RA_BF16 ? 2 : 4);
   cudaError_t e;
   if (q->dtype == RA_BF16) {
     const int dp = padded_dim(w.d);

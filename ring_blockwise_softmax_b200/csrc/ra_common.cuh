@@ -306,6 +306,7 @@ enum EpilogueMode : int {
 struct AttnWork {
   int B;          // batch
   int r_major;    // work-item order: 1 = query shards outermost (contiguous shards), 0 = blocks
+  int hgroup;     // heads per item group (the group's K/V is sized to stay resident in L2)
   int n_q;        // query tokens per shard
   int n_kv;       // key tokens per shard
   int H;          // heads

@@ -205,11 +205,18 @@ struct Item {
   long long pos_last;  // position of the item's last valid query row
 };
 
+// Items come in head groups of w.hgroup (batch, head) pairs, so the K/V the concurrently running
+// CTAs read stays in L2; inside a group the order is longest first with heads innermost.
 __device__ __forceinline__ void decode_item(const AttnWork& w, int idx, Item& it) {
   const int n_blk = (w.n_q + 255) / 256;
   const int bh_count = w.B * w.H;
-  const int bh = idx % bh_count;
-  const int rest = idx / bh_count;
+  const int per_head = n_blk * w.n_r;
+  const int hg = w.hgroup;
+  const int grp = idx / (hg * per_head);
+  const int local = idx - grp * hg * per_head;
+  const int heads = min(hg, bh_count - grp * hg);
+  const int bh = grp * hg + local % heads;
+  const int rest = local / heads;
   int ri, blk;
   if (w.r_major) {  // positions grow with the shard first (contiguous shards): longest first
     ri = w.n_r - 1 - rest / n_blk;
