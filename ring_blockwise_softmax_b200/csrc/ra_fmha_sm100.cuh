@@ -76,7 +76,7 @@ template <int DP, int EPI>
 struct RegSplit {
   static constexpr bool kAcc = (EPI == 2 || EPI == 3);
   static constexpr int kProd = 80;
-  static constexpr int kEpi = kAcc ? 80 : 64;
+  static constexpr int kEpi = kAcc ? 80 : (DP <= 64 ? 48 : 64);
   static constexpr int kSoftmax = ((65536 / 128 - kProd - kEpi) / 2) / 8 * 8;
   static_assert(2 * 128 * kSoftmax + 128 * kEpi + 128 * kProd <= 65536, "register split exceeds the launch");
 };
@@ -409,10 +409,33 @@ __device__ __forceinline__ void fmha_epilogue_row(const AttnWork& w, const Item&
   }
 }
 
-// p = 2^(s * scale_log2 - base) for the 128 scores of this row, packed to bf16 pairs and stored
-// to tensor memory; row sums accumulated in two packed fp32x2 chains.  EVERY > 0: one column pair
-// in EVERY goes to the FMA-pipe polynomial instead of the MUFU (only for tiles without masked
+// p = 2^(s * scale_log2 - base) for the 128 scores of this row, packed to bf16 pairs in pk (the
+// row of P_q); row sums accumulated in two packed fp32x2 chains.  EVERY > 0: one column pair in
+// EVERY goes to the FMA-pipe polynomial instead of the MUFU (only for tiles without masked
 // scores, see exp2_poly3).
+template <int EVERY>
+__device__ __forceinline__ void softmax_exp(const uint32_t (&sr)[4][32], float sl2, float base, uint32_t (&pk)[64],
+                                            float2 (&rs)[2]) {
+  const float2 sc = make_float2(sl2, sl2);
+  const float2 nb = make_float2(-base, -base);
+#pragma unroll
+  for (int e = 0; e < 64; ++e) {
+    const float2 x = __ffma2_rn(
+        make_float2(__uint_as_float(sr[e >> 4][(2 * e) & 31]), __uint_as_float(sr[e >> 4][(2 * e + 1) & 31])), sc, nb);
+    float2 p;
+    if (EVERY > 0 && (e % (EVERY > 0 ? EVERY : 1)) == (EVERY > 0 ? EVERY : 1) - 1) {
+      p = exp2_poly3_x2(x);
+    } else {
+      p.x = ex2_approx(x.x);
+      p.y = ex2_approx(x.y);
+    }
+    rs[e & 1] = __fadd2_rn(rs[e & 1], p);
+    pk[e] = pack_bf16x2(p.x, p.y);
+  }
+}
+
+// As softmax_exp, but each 16-pair chunk of P_q goes to tensor memory as soon as it is computed
+// (fewer live registers; used where P_q's columns are known to be free before the exponentials).
 template <int EVERY>
 __device__ __forceinline__ void softmax_exp_store(const uint32_t (&sr)[4][32], float sl2, float base, uint32_t p_addr,
                                                   float2 (&rs)[2]) {
@@ -798,19 +821,37 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
         const float base = (m_new == -INFINITY) ? 0.f : m_new;
-        // P_q in its own columns is free once the previous PV_q has read it; the O rescale
-        // needs that PV to have landed too.
         const bool any_rescale = __any_sync(0xffffffffu, rescale);
-        if ((C::P_SEP || any_rescale) && c > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + q, (c - 1) & 1, ctl, 0x302));
-          if (!ok) break;
-          tc_fence_after();
-        }
         float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // packed row sums
-        if (masked || kEmuEvery == 0)
-          softmax_exp_store<0>(sr, sl2, base, p_addr, rsp);
-        else
-          softmax_exp_store<kEmuEvery>(sr, sl2, base, p_addr, rsp);
+        if (C::P_SEP) {
+          // P_q has its own columns, which the previous PV_q may still be reading.  The
+          // exponentials are computed into registers first, so by the time of this wait that PV
+          // has almost always landed.
+          uint32_t pk[64];
+          if (masked || kEmuEvery == 0)
+            softmax_exp<0>(sr, sl2, base, pk, rsp);
+          else
+            softmax_exp<kEmuEvery>(sr, sl2, base, pk, rsp);
+          if (c > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + q, (c - 1) & 1, ctl, 0x302));
+            if (!ok) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) tmem_st16(p_addr + cc * 16, pk + cc * 16);
+        } else {
+          // P_q over S_q: those columns are free once S_q is loaded (the next QK_q waits for this
+          // PV_q); only the O rescale needs the previous PV_q to have landed.
+          if (any_rescale && c > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + q, (c - 1) & 1, ctl, 0x302));
+            if (!ok) break;
+            tc_fence_after();
+          }
+          if (masked || kEmuEvery == 0)
+            softmax_exp_store<0>(sr, sl2, base, p_addr, rsp);
+          else
+            softmax_exp_store<kEmuEvery>(sr, sl2, base, p_addr, rsp);
+        }
         if (any_rescale) {
 #pragma unroll
           for (int cc = 0; cc < DP / 32; ++cc) {
