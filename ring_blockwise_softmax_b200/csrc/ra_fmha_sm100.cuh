@@ -63,7 +63,7 @@ struct FmhaCfg {
   static constexpr int P_COL0 = P_SEP ? 384 : 0;
   static constexpr int P_STRIDE = P_SEP ? 64 : 128;
   static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * STAGES);
-  static constexpr int NBAR = 3 + 3 * STAGES + 7 * 2;
+  static constexpr int NBAR = 3 + 3 * STAGES + 8 * 2;
   static constexpr int STATS_BYTES = 2 * 128 * 8;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES;
   static constexpr int THREADS = 512;
@@ -80,6 +80,13 @@ struct RegSplit {
   static constexpr int kSoftmax = ((65536 / 128 - kProd - kEpi) / 2) / 8 * 8;
   static_assert(2 * 128 * kSoftmax + 128 * kEpi + 128 * kProd <= 65536, "register split exceeds the launch");
 };
+
+// Exponential phases of the two softmax warpgroups strictly alternate (tile 0, tile 1, tile 0, ...)
+// so that each runs alone on the MUFU while the other waits, loads S and stores P.
+#ifndef RA_EXP_ALTERNATE
+#define RA_EXP_ALTERNATE 0
+#endif
+constexpr bool kExpAlternate = RA_EXP_ALTERNATE != 0;
 
 #ifndef RA_EMU_EVERY
 #define RA_EMU_EVERY 0
@@ -490,7 +497,8 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_o_empty = bar_o_full + 2;           // [2]
   uint64_t* bar_stats = bar_o_empty + 2;            // [2]
   uint64_t* bar_s_free = bar_stats + 2;             // [2] softmax has loaded S_q into registers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s_free + 2);
+  uint64_t* bar_tok = bar_s_free + 2;               // [2] softmax q may start its exponentials
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tok + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* stats = reinterpret_cast<float2*>(tmem_slot + 4);  // [2][128] (m_used, l_sum)
 
@@ -515,6 +523,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(bar_o_empty + q, 128);
       mbar_init(bar_stats + q, 128);
       mbar_init(bar_s_free + q, 128);
+      mbar_init(bar_tok + q, 4);  // one arrival per warp of the other softmax warpgroup
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -823,6 +832,12 @@ __global__ void __launch_bounds__(512, 1)
         const float base = (m_new == -INFINITY) ? 0.f : m_new;
         const bool any_rescale = __any_sync(0xffffffffu, rescale);
         float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // packed row sums
+        // Turn to use the MUFU: tile 0's c-th exponential phase follows tile 1's (c-1)-th, tile 1's
+        // c-th follows tile 0's c-th.  Both warpgroups walk the same tiles, so the turns match.
+        if (kExpAlternate && (q == 1 || c > 0)) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_tok + q, static_cast<uint32_t>(q == 0 ? c - 1 : c) & 1, ctl, 0x304));
+          if (!ok) break;
+        }
         if (C::P_SEP) {
           // P_q has its own columns, which the previous PV_q may still be reading.  The
           // exponentials are computed into registers first, so by the time of this wait that PV
@@ -832,6 +847,10 @@ __global__ void __launch_bounds__(512, 1)
             softmax_exp<0>(sr, sl2, base, pk, rsp);
           else
             softmax_exp<kEmuEvery>(sr, sl2, base, pk, rsp);
+          if (kExpAlternate) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tok + (q ^ 1));
+          }
           if (c > 0) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + q, (c - 1) & 1, ctl, 0x302));
             if (!ok) break;
@@ -851,6 +870,10 @@ __global__ void __launch_bounds__(512, 1)
             softmax_exp_store<0>(sr, sl2, base, p_addr, rsp);
           else
             softmax_exp_store<kEmuEvery>(sr, sl2, base, p_addr, rsp);
+          if (kExpAlternate) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tok + (q ^ 1));
+          }
         }
         if (any_rescale) {
 #pragma unroll
