@@ -63,7 +63,7 @@ struct FmhaCfg {
   static constexpr int P_COL0 = P_SEP ? 384 : 0;
   static constexpr int P_STRIDE = P_SEP ? 64 : 128;
   static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * STAGES);
-  static constexpr int NBAR = 3 + 3 * STAGES + 8 * 2;
+  static constexpr int NBAR = 3 + 3 * STAGES + 7 * 2;
   static constexpr int STATS_BYTES = 2 * 128 * 8;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES;
   static constexpr int THREADS = 512;
@@ -80,13 +80,6 @@ struct RegSplit {
   static constexpr int kSoftmax = ((65536 / 128 - kProd - kEpi) / 2) / 8 * 8;
   static_assert(2 * 128 * kSoftmax + 128 * kEpi + 128 * kProd <= 65536, "register split exceeds the launch");
 };
-
-// Exponential phases of the two softmax warpgroups strictly alternate (tile 0, tile 1, tile 0, ...)
-// so that each runs alone on the MUFU while the other waits, loads S and stores P.
-#ifndef RA_EXP_ALTERNATE
-#define RA_EXP_ALTERNATE 0
-#endif
-constexpr bool kExpAlternate = RA_EXP_ALTERNATE != 0;
 
 #ifndef RA_EMU_EVERY
 #define RA_EMU_EVERY 0
@@ -176,6 +169,39 @@ __device__ __forceinline__ bool mbar_wait_issuer(uint64_t* bar, uint32_t parity,
       if (mbar_test_wait(bar, parity)) return true;
     if (*ctl.abort) return false;
     if (globaltimer_ns() - t0 > ctl.limit_ns) {
+      atomicOr(ctl.status, kDevStatusTimeout);
+      atomicCAS(ctl.status + 1, 0u, site);
+      *ctl.abort = 1;
+      __threadfence_block();
+      return false;
+    }
+  }
+}
+
+// Wait used by the MMA issuers for everything one MMA group needs: up to three (barrier, parity)
+// pairs (nullptr = none).  Each poll tests every pair not yet seen complete back to back, so the
+// latencies of the tests (a few hundred cycles even on a completed phase) overlap instead of
+// adding up.  Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_all_issuer(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
+                                                     uint32_t p2, const WaitCtl& ctl, unsigned site) {
+  bool d0 = b0 == nullptr, d1 = b1 == nullptr, d2 = b2 == nullptr;
+  auto poll = [&]() -> bool {
+    const bool t0 = d0 || mbar_test_wait(b0, p0);
+    const bool t1 = d1 || mbar_test_wait(b1, p1);
+    const bool t2 = d2 || mbar_test_wait(b2, p2);
+    d0 = t0;
+    d1 = t1;
+    d2 = t2;
+    return t0 && t1 && t2;
+  };
+  if (poll()) return true;
+  const uint64_t start = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+      if (poll()) return true;
+    if (*ctl.abort) return false;
+    if (globaltimer_ns() - start > ctl.limit_ns) {
       atomicOr(ctl.status, kDevStatusTimeout);
       atomicCAS(ctl.status + 1, 0u, site);
       *ctl.abort = 1;
@@ -416,17 +442,17 @@ __device__ __forceinline__ void fmha_epilogue_row(const AttnWork& w, const Item&
   }
 }
 
-// p = 2^(s * scale_log2 - base) for the 128 scores of this row, packed to bf16 pairs in pk (the
-// row of P_q); row sums accumulated in two packed fp32x2 chains.  EVERY > 0: one column pair in
+// p = 2^(s * scale_log2 - base) for the scores of column pairs [E0, E1) of this row, packed to
+// bf16 pairs in pk (the row of P_q); row sums accumulated in two packed fp32x2 chains.  EVERY > 0: one column pair in
 // EVERY goes to the FMA-pipe polynomial instead of the MUFU (only for tiles without masked
 // scores, see exp2_poly3).
-template <int EVERY>
+template <int EVERY, int E0 = 0, int E1 = 64>
 __device__ __forceinline__ void softmax_exp(const uint32_t (&sr)[4][32], float sl2, float base, uint32_t (&pk)[64],
                                             float2 (&rs)[2]) {
   const float2 sc = make_float2(sl2, sl2);
   const float2 nb = make_float2(-base, -base);
 #pragma unroll
-  for (int e = 0; e < 64; ++e) {
+  for (int e = E0; e < E1; ++e) {
     const float2 x = __ffma2_rn(
         make_float2(__uint_as_float(sr[e >> 4][(2 * e) & 31]), __uint_as_float(sr[e >> 4][(2 * e + 1) & 31])), sc, nb);
     float2 p;
@@ -497,8 +523,7 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_o_empty = bar_o_full + 2;           // [2]
   uint64_t* bar_stats = bar_o_empty + 2;            // [2]
   uint64_t* bar_s_free = bar_stats + 2;             // [2] softmax has loaded S_q into registers
-  uint64_t* bar_tok = bar_s_free + 2;               // [2] softmax q may start its exponentials
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tok + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s_free + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* stats = reinterpret_cast<float2*>(tmem_slot + 4);  // [2][128] (m_used, l_sum)
 
@@ -523,7 +548,6 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(bar_o_empty + q, 128);
       mbar_init(bar_stats + q, 128);
       mbar_init(bar_s_free + q, 128);
-      mbar_init(bar_tok + q, 4);  // one arrival per warp of the other softmax warpgroup
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -638,10 +662,9 @@ __global__ void __launch_bounds__(512, 1)
           const long long gj = g + j;
           const bool has_next = j + 1 < n;
           for (int q = 0; q < 2 && ok; ++q) {
-            ok = mbar_wait_issuer(bar_p_full + q, static_cast<uint32_t>(gj) & 1, ctl, 0x205) &&
-                 (q == 1 || mbar_wait_issuer(bar_v_full + gj % C::STAGES, static_cast<uint32_t>(gj / C::STAGES) & 1, ctl,
-                                             0x206)) &&
-                 (j > 0 || it_all == 0 || mbar_wait_issuer(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x207));
+            ok = mbar_wait_all_issuer(bar_p_full + q, static_cast<uint32_t>(gj) & 1,
+                                      q == 1 ? nullptr : bar_v_full + gj % C::STAGES, static_cast<uint32_t>(gj / C::STAGES) & 1,
+                                      (j > 0 || it_all == 0) ? nullptr : bar_o_empty + q, (it_all - 1) & 1, ctl, 0x205);
             if (!ok) break;
             tc_fence_after();
             fmha_issue_pv<C>(db, tmem + C::O_COL0 + C::O_STRIDE * q, tmem + C::P_COL0 + C::P_STRIDE * q,
@@ -649,9 +672,9 @@ __global__ void __launch_bounds__(512, 1)
             mma_commit(bar_pv_done + q);
             if (has_next) {
               const long long gn = gj + 1;
-              ok = (q == 1 || mbar_wait_issuer(bar_k_full + gn % C::STAGES, static_cast<uint32_t>(gn / C::STAGES) & 1,
-                                               ctl, 0x209)) &&
-                   mbar_wait_issuer(bar_pv_done + q, static_cast<uint32_t>(gj) & 1, ctl, 0x20a);
+              ok = mbar_wait_all_issuer(bar_pv_done + q, static_cast<uint32_t>(gj) & 1,
+                                        q == 1 ? nullptr : bar_k_full + gn % C::STAGES,
+                                        static_cast<uint32_t>(gn / C::STAGES) & 1, nullptr, 0, ctl, 0x209);
               if (!ok) break;
               tc_fence_after();
               fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
@@ -702,14 +725,9 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = true;
       auto qk = [&](long long gk, bool last_of_item) -> bool {
         // S_q must be free: the previous QK's S consumed (own P columns) or its PV done (P over S).
-        if (cq > 0) {
-          if (C::P_SEP) {
-            if (!mbar_wait_issuer(bar_s_free + q, (cq - 1) & 1, ctl, 0x202)) return false;
-          } else {
-            if (!mbar_wait_issuer(bar_pv_done + q, (cq - 1) & 1, ctl, 0x203)) return false;
-          }
-        }
-        if (!mbar_wait_issuer(bar_k_full + gk % C::STAGES, static_cast<uint32_t>(gk / C::STAGES) & 1, ctl, 0x204))
+        if (!mbar_wait_all_issuer(cq > 0 ? (C::P_SEP ? bar_s_free + q : bar_pv_done + q) : nullptr, (cq - 1) & 1,
+                                  bar_k_full + gk % C::STAGES, static_cast<uint32_t>(gk / C::STAGES) & 1, nullptr, 0,
+                                  ctl, 0x202))
           return false;
         tc_fence_after();
         fmha_issue_qk<C>(db, d_s, q_addr, k_base + static_cast<int>(gk % C::STAGES) * C::TILE_BYTES, idesc_qk);
@@ -729,9 +747,9 @@ __global__ void __launch_bounds__(512, 1)
           for (int j = 0; ok && j < n; ++j) {
             const long long gj = g + j;
             if (C::P_SEP && j + 1 < n && !(ok = qk(gj + 1, j + 2 == n))) break;
-            ok = mbar_wait_issuer(bar_p_full + q, cpv & 1, ctl, 0x205) &&
-                 mbar_wait_issuer(bar_v_full + gj % C::STAGES, static_cast<uint32_t>(gj / C::STAGES) & 1, ctl, 0x206) &&
-                 (j > 0 || it_all == 0 || mbar_wait_issuer(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x207));
+            ok = mbar_wait_all_issuer(bar_p_full + q, cpv & 1, bar_v_full + gj % C::STAGES,
+                                      static_cast<uint32_t>(gj / C::STAGES) & 1,
+                                      (j > 0 || it_all == 0) ? nullptr : bar_o_empty + q, (it_all - 1) & 1, ctl, 0x206);
             if (!ok) break;
             tc_fence_after();
             fmha_issue_pv<C>(db, d_o, p_t, v_base + static_cast<int>(gj % C::STAGES) * C::TILE_BYTES, idesc_pv,
@@ -768,6 +786,9 @@ __global__ void __launch_bounds__(512, 1)
     const float sl2 = w.scale_log2;
     int it_all = 0, c = 0;
     bool ok = true;
+    // Barrier tests issued ahead of their use: a test costs a few hundred cycles even when the
+    // phase is complete, so it is issued while the exponentials run and its result read later.
+    bool s_seen = false;  // S_q of tile c already seen complete
     for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
         const int idx = item_of_cta(k);
         if (idx >= n_items) continue;
@@ -784,8 +805,11 @@ __global__ void __launch_bounds__(512, 1)
           cur_s = wk.s;
           row_lim = row_ok ? visible_key_limit(w, pos_q, wk.s) : w.n_kv;
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + q, c & 1, ctl, 0x301));
-        if (!ok) break;
+        if (!__all_sync(0xffffffffu, s_seen)) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + q, c & 1, ctl, 0x301));
+          if (!ok) break;
+        }
+        s_seen = false;
         tc_fence_after();
         uint32_t sr[4][32];
 #pragma unroll
@@ -832,30 +856,27 @@ __global__ void __launch_bounds__(512, 1)
         const float base = (m_new == -INFINITY) ? 0.f : m_new;
         const bool any_rescale = __any_sync(0xffffffffu, rescale);
         float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // packed row sums
-        // Turn to use the MUFU: tile 0's c-th exponential phase follows tile 1's (c-1)-th, tile 1's
-        // c-th follows tile 0's c-th.  Both warpgroups walk the same tiles, so the turns match.
-        if (kExpAlternate && (q == 1 || c > 0)) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar_tok + q, static_cast<uint32_t>(q == 0 ? c - 1 : c) & 1, ctl, 0x304));
-          if (!ok) break;
-        }
         if (C::P_SEP) {
           // P_q has its own columns, which the previous PV_q may still be reading.  The
           // exponentials are computed into registers first, so by the time of this wait that PV
           // has almost always landed.
           uint32_t pk[64];
-          if (masked || kEmuEvery == 0)
-            softmax_exp<0>(sr, sl2, base, pk, rsp);
-          else
-            softmax_exp<kEmuEvery>(sr, sl2, base, pk, rsp);
-          if (kExpAlternate) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tok + (q ^ 1));
+          bool pv_seen;
+          if (masked || kEmuEvery == 0) {
+            softmax_exp<0, 0, 32>(sr, sl2, base, pk, rsp);
+            pv_seen = c == 0 || mbar_test_wait(bar_pv_done + q, (c - 1) & 1);
+            softmax_exp<0, 32, 64>(sr, sl2, base, pk, rsp);
+          } else {
+            softmax_exp<kEmuEvery, 0, 32>(sr, sl2, base, pk, rsp);
+            pv_seen = c == 0 || mbar_test_wait(bar_pv_done + q, (c - 1) & 1);
+            softmax_exp<kEmuEvery, 32, 64>(sr, sl2, base, pk, rsp);
           }
-          if (c > 0) {
+          s_seen = mbar_test_wait(bar_s_full + q, (c + 1) & 1);  // the next QK_q, issued at s_free
+          if (!__all_sync(0xffffffffu, pv_seen)) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + q, (c - 1) & 1, ctl, 0x302));
             if (!ok) break;
-            tc_fence_after();
           }
+          tc_fence_after();
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) tmem_st16(p_addr + cc * 16, pk + cc * 16);
         } else {
@@ -870,10 +891,6 @@ __global__ void __launch_bounds__(512, 1)
             softmax_exp_store<0>(sr, sl2, base, p_addr, rsp);
           else
             softmax_exp_store<kEmuEvery>(sr, sl2, base, p_addr, rsp);
-          if (kExpAlternate) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tok + (q ^ 1));
-          }
         }
         if (any_rescale) {
 #pragma unroll
