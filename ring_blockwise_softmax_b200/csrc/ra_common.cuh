@@ -344,12 +344,23 @@ struct AttnWork {
 
 // Number of keys u in [0, n_kv) of shard s that are visible to a query at global position
 // pos_q: all of them if not causal, else those with k_off + s*k_sstep + u*k_ustride <= pos_q.
+// (k_ustride >= 1.)  The quotient is taken in 32 bits whenever the operands fit: a 64-bit division
+// is a long dependent instruction sequence, and every role of the attention kernel evaluates this
+// at each work item's start, on the item's critical path.
 __host__ __device__ __forceinline__ int visible_key_limit(const AttnWork& w, long long pos_q, int s) {
   if (!w.causal) return w.n_kv;
   const long long base = w.k_off + static_cast<long long>(s) * w.k_sstep;
   if (pos_q < base) return 0;
-  const long long lim = (pos_q - base) / w.k_ustride + 1;
-  return lim < w.n_kv ? static_cast<int>(lim) : w.n_kv;
+  const unsigned long long diff = static_cast<unsigned long long>(pos_q - base);
+  const unsigned long long stride = static_cast<unsigned long long>(w.k_ustride);
+  unsigned long long quot;
+  if (stride == 1)
+    quot = diff;
+  else if (((diff | stride) >> 32) == 0)
+    quot = static_cast<unsigned>(diff) / static_cast<unsigned>(stride);
+  else
+    quot = diff / stride;
+  return quot < static_cast<unsigned long long>(w.n_kv) ? static_cast<int>(quot) + 1 : w.n_kv;
 }
 
 __host__ __device__ __forceinline__ int ring_kv_shard(const AttnWork& w, int r) {
