@@ -251,6 +251,24 @@ ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::A
   if (w_in.B > 65535 || w_in.H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
   ra::AttnWork w = w_in;
   w.hgroup = heads_per_group(w, q->dtype == RA_BF16 ? 2 : 4);
+  {
+    // Launch-time fast dividers for the kernels' index arithmetic (all operands stay below 2^31).
+    const long long n_blk = (static_cast<long long>(w.n_q) + 255) / 256;
+    const long long per_group = static_cast<long long>(w.hgroup) * n_blk * w.n_r;
+    const long long bh = static_cast<long long>(w.B) * w.H;
+    if (per_group * ((bh + w.hgroup - 1) / w.hgroup) > 2147483647LL || w.k_ustride > 2147483647LL ||
+        w.ring_step < 0 || w.ring_step + n_steps > 2 * w.P)
+      return fail(RA_ERR_UNSUPPORTED, "problem too large for 32-bit work-item indices");
+    const long long hg_last = bh - (bh - 1) / w.hgroup * w.hgroup;
+    w.fd_grp = ra::make_fastdiv(static_cast<unsigned>(per_group));
+    w.fd_hg = ra::make_fastdiv(static_cast<unsigned>(w.hgroup));
+    w.fd_hg_last = ra::make_fastdiv(static_cast<unsigned>(hg_last));
+    w.fd_nblk = ra::make_fastdiv(static_cast<unsigned>(n_blk));
+    w.fd_nr = ra::make_fastdiv(static_cast<unsigned>(w.n_r));
+    w.fd_H = ra::make_fastdiv(static_cast<unsigned>(w.H));
+    w.fd_P = ra::make_fastdiv(static_cast<unsigned>(w.P));
+    w.fd_kus = ra::make_fastdiv(static_cast<unsigned>(w.k_ustride));
+  }
   cudaError_t e;
   if (q->dtype == RA_BF16) {
     const int dp = padded_dim(w.d);

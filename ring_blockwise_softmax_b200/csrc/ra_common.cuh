@@ -303,6 +303,34 @@ enum EpilogueMode : int {
   kEpiAccOut = 3,  // merge with the fp32 accumulator and write the result to the output
 };
 
+// Division by a divisor fixed for the launch, as a multiply and shift (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994): with s = ceil(log2 d) and
+// m = ceil(2^(32+s) / d), floor(n / d) = (n * m) >> (32 + s) exactly for 0 <= n < 2^31 (the
+// rounding error n * (m * d - 2^(32+s)) / (d * 2^(32+s)) stays below 1/d).  The kernel's
+// per-item index arithmetic uses it because the hardware integer divide sequence goes through
+// the MUFU unit, which the softmax keeps saturated with exponentials.
+struct FastDiv {
+  unsigned long long m;
+  unsigned int d;
+  unsigned int s;
+};
+
+inline FastDiv make_fastdiv(unsigned int d) {  // host side; d >= 1
+  FastDiv f;
+  f.d = d;
+  f.s = 0;
+  while ((1ull << f.s) < d) ++f.s;
+  f.m = ((1ull << (32 + f.s)) + d - 1) / d;
+  return f;
+}
+
+__host__ __device__ __forceinline__ int fdiv(int n, const FastDiv& f) {  // 0 <= n < 2^31
+  return static_cast<int>((static_cast<unsigned long long>(n) * f.m) >> (32 + f.s));
+}
+__host__ __device__ __forceinline__ int fmod_(int n, const FastDiv& f) {
+  return n - fdiv(n, f) * static_cast<int>(f.d);
+}
+
 struct AttnWork {
   int B;          // batch
   int r_major;    // work-item order: 1 = query shards outermost (contiguous shards), 0 = blocks
@@ -340,13 +368,16 @@ struct AttnWork {
   long long al_sb, al_sh, al_rs, al_ts;
   unsigned long long wait_limit_ns;
   unsigned int* dev_status;
+  // Fast dividers (set at launch): items per head group, heads per group, heads of the last group,
+  // 256-row blocks per shard, query shards, heads, ring size, key position stride.
+  FastDiv fd_grp, fd_hg, fd_hg_last, fd_nblk, fd_nr, fd_H, fd_P, fd_kus;
 };
 
 // Number of keys u in [0, n_kv) of shard s that are visible to a query at global position
 // pos_q: all of them if not causal, else those with k_off + s*k_sstep + u*k_ustride <= pos_q.
-// (k_ustride >= 1.)  The quotient is taken in 32 bits whenever the operands fit: a 64-bit division
-// is a long dependent instruction sequence, and every role of the attention kernel evaluates this
-// at each work item's start, on the item's critical path.
+// (k_ustride >= 1.)  The quotient avoids the divide instruction sequence whenever the operands
+// fit: every role of the attention kernel evaluates this at each work item's start, on the item's
+// critical path.
 __host__ __device__ __forceinline__ int visible_key_limit(const AttnWork& w, long long pos_q, int s) {
   if (!w.causal) return w.n_kv;
   const long long base = w.k_off + static_cast<long long>(s) * w.k_sstep;
@@ -356,16 +387,16 @@ __host__ __device__ __forceinline__ int visible_key_limit(const AttnWork& w, lon
   unsigned long long quot;
   if (stride == 1)
     quot = diff;
-  else if (((diff | stride) >> 32) == 0)
-    quot = static_cast<unsigned>(diff) / static_cast<unsigned>(stride);
+  else if ((diff >> 31) == 0 && stride == w.fd_kus.d)
+    quot = static_cast<unsigned long long>(fdiv(static_cast<int>(diff), w.fd_kus));
   else
     quot = diff / stride;
   return quot < static_cast<unsigned long long>(w.n_kv) ? static_cast<int>(quot) + 1 : w.n_kv;
 }
 
-__host__ __device__ __forceinline__ int ring_kv_shard(const AttnWork& w, int r) {
-  int s = (r - w.ring_step) % w.P;
-  return s < 0 ? s + w.P : s;
+// (r - t) mod P for 0 <= r < P, 0 <= t < 2P (the launch keeps ring_step + steps <= 2P).
+__host__ __device__ __forceinline__ int ring_shard(const AttnWork& w, int r, int t) {
+  return fmod_(r - t + 2 * w.P, w.fd_P);
 }
 
 }  // namespace ra

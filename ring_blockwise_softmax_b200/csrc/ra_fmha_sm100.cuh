@@ -241,25 +241,29 @@ struct Item {
 // Items come in head groups of w.hgroup (batch, head) pairs, so the K/V the concurrently running
 // CTAs read stays in L2; inside a group the order is longest first with heads innermost.
 __device__ __forceinline__ void decode_item(const AttnWork& w, int idx, Item& it) {
-  const int n_blk = (w.n_q + 255) / 256;
+  // Index arithmetic with launch-time fast dividers only (no divide instructions).
+  const int n_blk = (w.n_q + 255) >> 8;
   const int bh_count = w.B * w.H;
   const int per_head = n_blk * w.n_r;
   const int hg = w.hgroup;
-  const int grp = idx / (hg * per_head);
+  const int grp = fdiv(idx, w.fd_grp);  // items per group = hg * per_head
   const int local = idx - grp * hg * per_head;
-  const int heads = min(hg, bh_count - grp * hg);
-  const int bh = grp * hg + local % heads;
-  const int rest = local / heads;
+  const bool last_grp = bh_count - grp * hg < hg;
+  const FastDiv& fh = last_grp ? w.fd_hg_last : w.fd_hg;
+  const int rest = fdiv(local, fh);
+  const int bh = grp * hg + (local - rest * static_cast<int>(fh.d));
   int ri, blk;
   if (w.r_major) {  // positions grow with the shard first (contiguous shards): longest first
-    ri = w.n_r - 1 - rest / n_blk;
-    blk = n_blk - 1 - rest % n_blk;
+    const int a = fdiv(rest, w.fd_nblk);
+    ri = w.n_r - 1 - a;
+    blk = n_blk - 1 - (rest - a * n_blk);
   } else {
-    blk = n_blk - 1 - rest / w.n_r;
-    ri = w.n_r - 1 - rest % w.n_r;
+    const int a = fdiv(rest, w.fd_nr);
+    blk = n_blk - 1 - a;
+    ri = w.n_r - 1 - (rest - a * w.n_r);
   }
-  it.b = bh / w.H;
-  it.h = bh % w.H;
+  it.b = fdiv(bh, w.fd_H);
+  it.h = bh - it.b * w.H;
   it.r = w.r_first + ri * w.r_step;
   it.t0 = blk * 256;
   it.rows_valid[0] = max(0, min(128, w.n_q - it.t0));
@@ -278,8 +282,7 @@ struct Walk {
 
 __device__ __forceinline__ bool walk_seek(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
   for (; k.step < n_steps; ++k.step) {
-    int s = (it.r - (w.ring_step + k.step)) % w.P;
-    if (s < 0) s += w.P;
+    const int s = ring_shard(w, it.r, w.ring_step + k.step);
     const int lim = visible_key_limit(w, it.pos_last, s);
     if (lim > 0) {
       k.s = s;
@@ -308,8 +311,7 @@ __device__ __forceinline__ bool walk_next(Walk& k, const AttnWork& w, const Item
 __device__ __forceinline__ int walk_count(const AttnWork& w, const Item& it, int n_steps) {
   int n = 0;
   for (int step = 0; step < n_steps; ++step) {
-    int s = (it.r - (w.ring_step + step)) % w.P;
-    if (s < 0) s += w.P;
+    const int s = ring_shard(w, it.r, w.ring_step + step);
     n += (visible_key_limit(w, it.pos_last, s) + FmhaCfg<32>::BN - 1) / FmhaCfg<32>::BN;
   }
   return n;
