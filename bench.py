@@ -47,6 +47,26 @@ def kernel_sources_hash() -> str:
     return h.hexdigest()
 
 
+# Exponential throughput of the MUFU unit: 16 ex2 per clock per SM (4 per sub-partition; a
+# micro-benchmark of the softmax's exponential loop on this GPU reaches ~3.8 per sub-partition).
+MUFU_EX2_PER_CLK_PER_SM = 16
+B200_SMS = 148
+
+
+def mufu_roofline(w, ms: float, world: int, clocks: dict):
+    """Second roofline for head dims <= 64, where the softmax exponentials (one per visible
+    query-key pair: algorithmic FLOPs / (4 d)) bind before the tensor core does.  Peak at the
+    median SM clock sampled during the timed region (the maximum clock when none was sampled)."""
+    if w.dtype != "bf16":
+        return None
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    exps = w.flops() / (4.0 * w.d)
+    achieved = world * exps / (ms * 1e-3) / 1e12
+    peak = world * MUFU_EX2_PER_CLK_PER_SM * B200_SMS * mhz * 1e6 / 1e12
+    return {"bound": "mufu", "achieved": achieved, "peak": peak, "unit": "Tex2/s", "frac": achieved / peak,
+            "note": "one exponential per visible (query, key) pair; peak = 16 ex2/clk/SM x 148 SMs x sampled SM clock"}
+
+
 def recorded_traffic(workload: str, schedule: str):
     """DRAM bytes per launch of the attention kernel from profiles/fmha_traffic.json, if that
     capture was taken of the current kernel sources on this workload and schedule; else None."""
@@ -399,6 +419,7 @@ def run_gpu(args, w):
                                                                                                   args.schedule),
                      "note": "algorithmic FLOPs (4*B*H*N^2*d, halved when causal) / summed duration of the step's "
                              f"{launches_per_step} serialised launches (CUDA events on the launch stream)"},
+        "mufu_roofline": mufu_roofline(w, ms, world, clocks.summary()),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
