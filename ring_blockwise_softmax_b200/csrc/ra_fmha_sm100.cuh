@@ -63,9 +63,10 @@ struct FmhaCfg {
   static constexpr int P_COL0 = P_SEP ? 384 : 0;
   static constexpr int P_STRIDE = P_SEP ? 64 : 128;
   static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * STAGES);
-  static constexpr int NBAR = 3 + 3 * STAGES + 7 * 2;
+  static constexpr int NBAR = 3 + 3 * STAGES + 9 * 2;
   static constexpr int STATS_BYTES = 2 * 128 * 8;
-  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES;
+  static constexpr int PLAN_BYTES = 2 * 48;
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES + PLAN_BYTES;
   static constexpr int THREADS = 512;
   static constexpr int D = DP;
 };
@@ -237,6 +238,16 @@ struct Item {
   long long pos0;      // global position of local query token 0 of shard r
   long long pos_last;  // position of the item's last valid query row
 };
+
+// A work item as the TMA producer publishes it to the other roles (decoded once per CTA).  Used
+// with P in its own tensor-memory columns (d <= 64), where item set-up sat on the critical path of
+// short causal items; the d = 128 roles decode items themselves (measured faster there).
+struct ItemPlan {
+  Item it;
+  int n;  // K/V tiles the item walks
+  int pad;
+};
+static_assert(sizeof(ItemPlan) == 48, "plan slot size");
 
 // Items come in head groups of w.hgroup (batch, head) pairs, so the K/V the concurrently running
 // CTAs read stays in L2; inside a group the order is longest first with heads innermost.
@@ -525,9 +536,12 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_o_empty = bar_o_full + 2;           // [2]
   uint64_t* bar_stats = bar_o_empty + 2;            // [2]
   uint64_t* bar_s_free = bar_stats + 2;             // [2] softmax has loaded S_q into registers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s_free + 2);
+  uint64_t* bar_plan_full = bar_s_free + 2;         // [2] item plan slot written
+  uint64_t* bar_plan_empty = bar_plan_full + 2;     // [2] item plan slot read by every consumer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_plan_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* stats = reinterpret_cast<float2*>(tmem_slot + 4);  // [2][128] (m_used, l_sum)
+  ItemPlan* plan = reinterpret_cast<ItemPlan*>(stats + 2 * 128);  // [2], slot = item sequence & 1
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -550,6 +564,9 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(bar_o_empty + q, 128);
       mbar_init(bar_stats + q, 128);
       mbar_init(bar_s_free + q, 128);
+      // Readers of a plan slot (d <= 64): each MMA issuer thread, 8 softmax warps, 4 epilogue warps.
+      mbar_init(bar_plan_full + q, 1);
+      mbar_init(bar_plan_empty + q, C::ISSUERS + 12);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -572,14 +589,24 @@ __global__ void __launch_bounds__(512, 1)
     setmaxnreg_dec<RegSplit<DP, EPI>::kProd>();
     if (warp == 12 && lane == 0) {
       // ================================================================ TMA producer
-      int it_q = 0;
+      int it_q = 0, it_seq = 0;
       long long g = 0;
       bool ok = true;
       for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
         const int idx = item_of_cta(k);
         if (idx >= n_items) continue;
+        // Publish the item's plan (decoded item and tile count) to the other roles.  The
+        // producer runs ahead of them, so this set-up leaves their critical path.
         Item it;
         decode_item(w, idx, it);
+        if (C::P_SEP) {
+          const int slot = it_seq & 1;
+          if (it_seq >= 2 && !mbar_wait(bar_plan_empty + slot, ((it_seq >> 1) - 1) & 1, ctl, 0x103)) break;
+          plan[slot].it = it;
+          plan[slot].n = walk_count(w, it, n_steps);
+          mbar_arrive(bar_plan_full + slot);
+          ++it_seq;
+        }
         Walk wk;
         bool has = walk_begin(wk, w, it, n_steps);
         if (!has) continue;
@@ -741,9 +768,9 @@ __global__ void __launch_bounds__(512, 1)
       for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
         const int idx = item_of_cta(k);
         if (idx >= n_items) continue;
-        Item it;
-        decode_item(w, idx, it);
-        const int n = walk_count(w, it, n_steps);
+        if (!(ok = mbar_wait_issuer(bar_plan_full + (it_all & 1), (it_all >> 1) & 1, ctl, 0x20b))) break;
+        const int n = plan[it_all & 1].n;
+        mbar_arrive(bar_plan_empty + (it_all & 1));
         if (n > 0) {
           ok = mbar_wait_issuer(bar_q_full, it_q & 1, ctl, 0x201) && qk(g, n == 1);
           for (int j = 0; ok && j < n; ++j) {
@@ -795,7 +822,15 @@ __global__ void __launch_bounds__(512, 1)
         const int idx = item_of_cta(k);
         if (idx >= n_items) continue;
       Item it;
-      decode_item(w, idx, it);
+      if (C::P_SEP) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_plan_full + (it_all & 1), (it_all >> 1) & 1, ctl, 0x305));
+        if (!ok) break;
+        it = plan[it_all & 1].it;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_plan_empty + (it_all & 1));
+      } else {
+        decode_item(w, idx, it);
+      }
       const bool row_ok = row < it.rows_valid[q];
       const long long pos_q = it.pos0 + static_cast<long long>(it.t0 + 128 * q + row) * w.q_tstride;
       float m_used = -INFINITY;  // running max of scaled scores, log2 units
@@ -938,9 +973,19 @@ __global__ void __launch_bounds__(512, 1)
         const int idx = item_of_cta(k);
         if (idx >= n_items) continue;
       Item it;
-      decode_item(w, idx, it);
-      Walk wk;
-      const bool has_o = walk_begin(wk, w, it, n_steps);
+      bool has_o;
+      if (C::P_SEP) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_plan_full + (it_all & 1), (it_all >> 1) & 1, ctl, 0x403));
+        if (!ok) break;
+        it = plan[it_all & 1].it;
+        has_o = plan[it_all & 1].n > 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_plan_empty + (it_all & 1));
+      } else {
+        decode_item(w, idx, it);
+        Walk wk;
+        has_o = walk_begin(wk, w, it, n_steps);
+      }
       for (int q = 0; q < 2; ++q) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_full + q, it_all & 1, ctl, 0x401) &&
                                          mbar_wait(bar_stats + q, it_all & 1, ctl, 0x402));
