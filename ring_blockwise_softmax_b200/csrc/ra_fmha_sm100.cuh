@@ -914,8 +914,7 @@ __global__ void __launch_bounds__(512, 1)
             if (!ok) break;
           }
           tc_fence_after();
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) tmem_st16(p_addr + cc * 16, pk + cc * 16);
+          tmem_st64(p_addr, pk);
         } else {
           // P_q over S_q: those columns are free once S_q is loaded (the next QK_q waits for this
           // PV_q); only the O rescale needs the previous PV_q to have landed.
