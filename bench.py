@@ -37,13 +37,16 @@ FMHA_SOURCES = ("ra_common.cuh", "ra_fmha_sm100.cuh", "ra_fmha_launch.cu")
 
 
 def kernel_sources_hash() -> str:
-    """sha256 over the attention kernel's sources (identifies the kernel build a capture is of)."""
+    """sha256 over the attention kernel's sources without blank and whole-line comment lines
+    (identifies the kernel code a capture is of; editing a comment does not invalidate it)."""
     import hashlib
 
     h = hashlib.sha256()
     for name in FMHA_SOURCES:
         with open(os.path.join(ROOT, "ring_blockwise_softmax_b200", "csrc", name), "rb") as fh:
-            h.update(name.encode() + b"\0" + fh.read())
+            code = [ln.strip() for ln in fh.read().splitlines()]
+        code = [ln for ln in code if ln and not ln.startswith(b"//")]
+        h.update(name.encode() + b"\0" + b"\n".join(code))
     return h.hexdigest()
 
 

@@ -16,21 +16,25 @@
 //   warps 0-3   softmax of query tile 0, thread i = row i = tensor-memory lane i
 //   warps 4-7   softmax of query tile 1
 //   warps 8-11  epilogue: normalise O, write O / LSE or LSE-merge into the accumulator
-//   warp 12     TMA producer: Q (two tiles) per item, then K_j / V_j into a STAGES-deep ring
-//   warps 13,14 MMA issuers, one thread per query tile: S_q = Q_q K_j^T (SS form),
-//               O_q += P_q V_j (TS form)
-// Both query tiles share every K/V tile (loaded once per 256 rows).  Each query tile has its own
-// MMA-issuing thread, so while one softmax warpgroup works on its S the tensor core runs the
-// other tile's PV and next QK; with P in its own columns (DP <= 64) the next QK_q starts as soon
-// as S_q is in registers.
+//   warp 12     TMA producer: Q (two tiles) per item, then K_j / V_j into a STAGES-deep ring;
+//               for DP <= 64 it also publishes each item's decoded plan (ItemPlan) to the others
+//   warps 13,14 MMA issuers, one thread per query tile (DP <= 64): S_q = Q_q K_j^T (SS form),
+//               O_q += P_q V_j (TS form); for DP = 128 one thread in warp 13 issues both tiles'
+//               MMAs in the fixed order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1)
+// Both query tiles share every K/V tile (loaded once per 256 rows).  With P in its own columns
+// (DP <= 64) the next QK_q starts as soon as S_q is in registers, so it overlaps this tile's
+// softmax.
 // Tensor memory (512 columns): S_0, S_1 (128 fp32 columns each), O_0, O_1 (DP columns each),
 // and P_0, P_1 (bf16 pairs, 64 columns each) in their own columns when DP <= 64, otherwise over
 // the first half of S_q (then S_q is rewritten only after PV_q has consumed P_q).
-// Registers are rebalanced with setmaxnreg (RegSplit): producer/MMA 80, epilogue 64 (80 when
-// merging), softmax the rest (176-184).
-// Part of the exponentials (1 in kEmuEvery column pairs of unmasked tiles) can run as a
-// polynomial on the FMA pipe to offload the MUFU unit (exp2_poly3).  The softmax arithmetic
-// uses packed fp32x2 instructions and three-input max.
+// Registers are rebalanced with setmaxnreg (RegSplit): producer/MMA 80, epilogue 48 (DP <= 64) or
+// 64 (80 when merging), softmax the rest (176-184).
+// Hand-offs: an issuer polls every barrier an MMA group needs in one loop, the softmax tests its
+// next barriers while its exponentials run, and work-item index arithmetic uses launch-time
+// multiply-shift dividers (an integer divide would queue behind the exponentials on the MUFU).
+// The softmax arithmetic uses packed fp32x2 instructions and three-input max.  A polynomial
+// exp2 on the FMA pipe (exp2_poly3) can take 1 in kEmuEvery column pairs of unmasked tiles; it
+// is off by default (measured slower).
 // Every wait is bounded; on a timeout all roles stop, tensor memory is freed and the kernel
 // returns with the device status word set.
 #pragma once
