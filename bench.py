@@ -237,8 +237,9 @@ class OracleSampler:
         # query rows drawn uniformly (seeded), so causal rows see N/2 keys on average
         rows = np.sort(self.rng.choice(w.N, size=min(self.rows, w.N), replace=False))
         pos = np.arange(w.N)
-        k = self.k[b, h].astype(np.float64)
-        v = self.v[b, h].astype(np.float64)
+        hk = oracle.kv_head(h, w.H, self.k.shape[1])  # K/V head (grouped-query K/V)
+        k = self.k[b, hk].astype(np.float64)
+        v = self.v[b, hk].astype(np.float64)
         oracle.attention_rows(self.q[b, h][rows].astype(np.float64), k, v, w.scale, rows, pos, w.causal)
         keys = (rows + 1).sum() if w.causal else self.rows * w.N
         self.flops += 4.0 * w.d * float(keys)
@@ -289,7 +290,9 @@ def run_reference(args, w):
 # the GPU arm
 # ---------------------------------------------------------------------------------------------
 def config_dict(w, args):
-    return {"workload": f"cfg{w.cfg}: {w.name}", "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+    name = w.name if w.H_kv is None else f"{w.name}, grouped-query K/V with {w.H_kv} heads"
+    return {"workload": f"cfg{w.cfg}: {name}", "B": w.B, "H": w.H, "H_kv": w.H_kv or w.H, "N": w.N, "d": w.d,
+            "causal": w.causal,
             "P": w.P, "layout": w.layout, "schedule": args.schedule,
             "l2": "flushed between timed steps (256 MiB write outside the events)",
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
@@ -409,6 +412,7 @@ def run_gpu(args, w):
     if rank != 0:
         return 0
     peak = peaks["bf16_tflops"]
+    traffic_key = f"cfg{w.cfg}" if w.H_kv is None else f"cfg{w.cfg}-kv{w.H_kv}"
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -418,7 +422,7 @@ def run_gpu(args, w):
         "pct_of_measured_bf16_peak": 100.0 * (value / world) / peak,
         "roofline": {"bound": "tensor", "kernel": "fmha_fwd_sm100", "achieved": value / world, "peak": peak,
                      "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s", "frac": (value / world) / peak,
-                     "traffic": args.traffic if args.traffic is not None else recorded_traffic(f"cfg{w.cfg}",
+                     "traffic": args.traffic if args.traffic is not None else recorded_traffic(traffic_key,
                                                                                                   args.schedule),
                      "note": "algorithmic FLOPs (4*B*H*N^2*d, halved when causal) / summed duration of the step's "
                              f"{launches_per_step} serialised launches (CUDA events on the launch stream)"},
@@ -451,6 +455,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-merge", action="store_true")
+    ap.add_argument("--kv-heads", type=int, default=None,
+                    help="grouped-query variant of the workload: K and V with this many heads (must divide H)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the attention kernel from an ncu capture of this build")
     args = ap.parse_args(argv)
@@ -459,6 +465,12 @@ def main(argv=None):
     from ring_blockwise_softmax_b200 import inputs as I
 
     w = I.WORKLOADS[args.config]
+    if args.kv_heads is not None:
+        if w.tabular is not None or args.kv_heads < 1 or w.H % args.kv_heads != 0:
+            raise SystemExit("--kv-heads must divide H and does not apply to the tabular workload")
+        import dataclasses
+
+        w = dataclasses.replace(w, H_kv=args.kv_heads)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

@@ -88,6 +88,13 @@ typedef struct {
   int64_t stride[4];
 } ra_tensor_t;
 
+/* Grouped-query / multi-query attention: in every call below, k and v may have H_kv heads
+ * instead of H (shape[1] = H_kv for both, H_kv dividing the query heads H of q).  Query head h
+ * then attends with K/V head h / (H / H_kv): consecutive groups of H / H_kv query heads share one
+ * K/V pair (vibe-research page, "MQA与GQA" section; H_kv = H is multi-head attention, H_kv = 1
+ * multi-query attention).  o and lse always have the H heads of q.  k and v with different head
+ * counts, or an H_kv that does not divide H, return RA_ERR_INVALID_ARG. */
+
 /* Global position of local token t: offset + t * stride (stride >= 1). */
 typedef struct {
   int64_t offset;
@@ -95,7 +102,7 @@ typedef struct {
 } ra_pos_t;
 
 /* Single full pass (ring with P = 1).
- * q [B,H,Nq,d]; k, v [B,H,Nk,d]; o [B,H,Nq,d] with o->dtype == q->dtype (bf16 in -> bf16 out,
+ * q [B,H,Nq,d]; k, v [B,H,Nk,d] (or [B,H_kv,Nk,d], see above); o [B,H,Nq,d] with o->dtype == q->dtype (bf16 in -> bf16 out,
  * fp32 in -> fp32 out); lse: fp32 [B,H,Nq] contiguous, may be NULL.  scale <= 0 selects
  * 1/sqrt(d).  causal != 0: query i and key j both sit at position = index (0-based), key j is
  * visible iff j <= i.  o must not overlap q, k or v. */
@@ -145,7 +152,8 @@ ra_status_t ra_ring_workspace_size(const ra_tensor_t* q, int P, int schedule, si
 /* Ring attention over P virtual sequence shards on one GPU (vibe-research page, "Ring
  * Attention" sequence diagram; intelliparadigm.com "Mosaic…", §3.2: KV blocks rotate, Q stays,
  * GPU r at step t uses the KV shard that started on GPU (r - t) mod P).
- * q, k, v [B,H,N,d] of one dtype with N % P == 0; the shards are views, nothing is copied:
+ * q, k, v [B,H,N,d] (k, v may have H_kv heads) of one dtype with N % P == 0; the shards are
+ * views, nothing is copied:
  *   layout RA_CONTIGUOUS: shard r = tokens [r*N/P, (r+1)*N/P);
  *   layout RA_STRIPED:    shard r = tokens r, r+P, r+2P, ... (token i on shard i mod P).
  * o [B,H,N,d] (dtype of q), lse fp32 [B,H,N] contiguous (may be NULL).  Positions are the

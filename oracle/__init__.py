@@ -14,7 +14,8 @@ Sources (web pages, cited by title and section):
         §3.4 (M-way merge through per-device (m_i, s_i)).
 * [VR]  vibe-research.pages.dev, "架构层解决方案 - Sparse Attention与Ring Attention":
         "Ring Attention" section, the blockwise softmax identity and the ring
-        sequence diagram (KV blocks rotate, each node accumulates).
+        sequence diagram (KV blocks rotate, each node accumulates); "MQA与GQA"
+        section (query-head groups sharing one K/V head).
 * [KK]  git.kang-kang.com, "注意力机制演进": timeline (Striped Attention),
         "FlashAttention" data-flow figure, "Ring Attention" figure.
 * [FA]  intelliparadigm.com, "深度学习注意力机制优化与FlashAttention实践":
@@ -43,5 +44,6 @@ from .fp64 import (  # noqa: F401
     merge_many,
     ring_attention,
     score_matrix_bytes,
+    kv_head,
 )
 from .sampling import sample_rows  # noqa: F401

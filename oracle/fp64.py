@@ -239,3 +239,16 @@ def ring_attention(q, k, v, P: int, layout: str, causal: bool, scale: float):
 def score_matrix_bytes(n_tokens: int, bytes_per_element: int) -> int:
     """Bytes of one materialised N x N score matrix ([FA] §2.2, [MO] §2.1)."""
     return int(n_tokens) * int(n_tokens) * int(bytes_per_element)
+
+
+def kv_head(h: int, n_heads: int, n_kv_heads: int) -> int:
+    """The key/value head that query head ``h`` attends with when ``n_kv_heads`` K/V heads serve
+    ``n_heads`` query heads ([VR] "MQA与GQA" section: the query heads are split into groups, each
+    group sharing one key/value pair; n_kv_heads = n_heads is multi-head attention, 1 is
+    multi-query attention).  Groups are consecutive query heads, as in the section's 32Q/8KV
+    figure where query heads 1-4 share K/V head 1."""
+    if n_kv_heads < 1 or n_heads % n_kv_heads != 0:
+        raise ValueError("the number of K/V heads must divide the number of query heads")
+    if not 0 <= h < n_heads:
+        raise ValueError("query head out of range")
+    return h // (n_heads // n_kv_heads)

@@ -235,7 +235,9 @@ struct Maps {
 // Heads per work-item group: the largest divisor of B*H (equal groups keep the longest-first
 // balance inside each group) whose K and V, all shards, fit in ~80 MiB of the 126 MB L2.
 int heads_per_group(const ra::AttnWork& w, int elem_bytes) {
-  const double kv_bytes = 2.0 * static_cast<double>(w.n_kv) * w.P * w.d * elem_bytes;
+  // K and V bytes per query head (query heads that share a K/V head share its bytes in L2).
+  const int qpk = (w.H_kv > 0 && w.H % w.H_kv == 0) ? w.H / w.H_kv : 1;
+  const double kv_bytes = 2.0 * static_cast<double>(w.n_kv) * w.P * w.d * elem_bytes / qpk;
   const double budget = 80.0 * 1024 * 1024;
   const long long bh = static_cast<long long>(w.B) * w.H;
   long long hg_max = static_cast<long long>(budget / (kv_bytes > 1.0 ? kv_bytes : 1.0));
@@ -250,6 +252,7 @@ ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::A
                              int sms, cudaStream_t stream) {
   if (w_in.B > 65535 || w_in.H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
   ra::AttnWork w = w_in;
+  if (w.H_kv == 0) w.H_kv = w.H;
   w.hgroup = heads_per_group(w, q->dtype == RA_BF16 ? 2 : 4);
   {
     // Launch-time fast dividers for the kernels' index arithmetic (all operands stay below 2^31).
@@ -268,6 +271,8 @@ ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::A
     w.fd_H = ra::make_fastdiv(static_cast<unsigned>(w.H));
     w.fd_P = ra::make_fastdiv(static_cast<unsigned>(w.P));
     w.fd_kus = ra::make_fastdiv(static_cast<unsigned>(w.k_ustride));
+    if (w.H_kv < 1 || w.H % w.H_kv != 0) return fail(RA_ERR_INVALID_ARG, "H_kv must divide H");
+    w.fd_qpk = ra::make_fastdiv(static_cast<unsigned>(w.H / w.H_kv));
   }
   cudaError_t e;
   if (q->dtype == RA_BF16) {
@@ -300,6 +305,7 @@ void set_operand_ptrs(ra::AttnWork& w, const ra_tensor_t* q, const ra_tensor_t* 
   w.q = q->data;
   w.k = k->data;
   w.v = v->data;
+  w.H_kv = static_cast<int>(k->shape[1]);
   w.q_sb = q->stride[0];
   w.q_sh = q->stride[1];
   w.q_rs = shard_rows * q->stride[2];
@@ -320,9 +326,11 @@ ra_status_t check_qkv(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tenso
   if ((st = check_tensor(k, "k")) != RA_OK) return st;
   if ((st = check_tensor(v, "v")) != RA_OK) return st;
   if (k->dtype != q->dtype || v->dtype != q->dtype) return fail(RA_ERR_INVALID_ARG, "q, k, v must share one dtype");
-  if (k->shape[0] != q->shape[0] || v->shape[0] != q->shape[0] || k->shape[1] != q->shape[1] ||
-      v->shape[1] != q->shape[1])
-    return fail(RA_ERR_INVALID_ARG, "q, k, v must agree on B and H");
+  if (k->shape[0] != q->shape[0] || v->shape[0] != q->shape[0])
+    return fail(RA_ERR_INVALID_ARG, "q, k, v must agree on B");
+  if (v->shape[1] != k->shape[1] || k->shape[1] < 1 || q->shape[1] % k->shape[1] != 0)
+    return fail(RA_ERR_INVALID_ARG, "k and v must have the same number of heads H_kv, and H_kv must divide the "
+                                    "query heads H (H_kv = H: multi-head, 1: multi-query, else grouped-query)");
   if (k->shape[3] != q->shape[3] || v->shape[3] != q->shape[3])
     return fail(RA_ERR_INVALID_ARG, "q, k, v must share the head dim");
   if (v->shape[2] != k->shape[2]) return fail(RA_ERR_INVALID_ARG, "k and v must have the same number of keys");

@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(128)
   const int tile = blockIdx.x % w.n_q_tiles;
   const int r = w.r_first + (blockIdx.x / w.n_q_tiles) * w.r_step;
   const int h = blockIdx.y;
+  const int hk = h / (w.H / w.H_kv);  // K/V head of this query head
   const int b = blockIdx.z;
   const int row = threadIdx.x >> 1;
   const int half = threadIdx.x & 1;
@@ -67,8 +68,8 @@ __global__ void __launch_bounds__(128)
         const int kr = e / DP, c = e % DP;
         const int u = u0 + kr;
         const bool in = (u < w.n_kv) && (c < w.d);
-        sk[kr][c] = in ? kg[b * w.k_sb + h * w.k_sh + s * w.k_rs + static_cast<long long>(u) * w.k_ts + c] : 0.f;
-        sv[kr][c] = in ? vg[b * w.v_sb + h * w.v_sh + s * w.v_rs + static_cast<long long>(u) * w.v_ts + c] : 0.f;
+        sk[kr][c] = in ? kg[b * w.k_sb + hk * w.k_sh + s * w.k_rs + static_cast<long long>(u) * w.k_ts + c] : 0.f;
+        sv[kr][c] = in ? vg[b * w.v_sb + hk * w.v_sh + s * w.v_rs + static_cast<long long>(u) * w.v_ts + c] : 0.f;
       }
       __syncthreads();
       float sc[kSimtKeys];

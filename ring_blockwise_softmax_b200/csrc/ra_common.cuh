@@ -346,7 +346,8 @@ struct AttnWork {
   int hgroup;     // heads per item group (the group's K/V is sized to stay resident in L2)
   int n_q;        // query tokens per shard
   int n_kv;       // key tokens per shard
-  int H;          // heads
+  int H;          // heads (of Q, O and LSE)
+  int H_kv;       // heads of K and V: query head h reads K/V head h / (H / H_kv) (GQA; MQA: 1)
   int d;          // head dim
   int P;          // shards in the ring (1 for a single pass / explicit partial)
   int n_q_tiles;  // ceil(n_q / 128) (tensor-core path) or ceil(n_q / rows per CTA)
@@ -380,6 +381,7 @@ struct AttnWork {
   // Fast dividers (set at launch): items per head group, heads per group, heads of the last group,
   // 256-row blocks per shard, query shards, heads, ring size, key position stride.
   FastDiv fd_grp, fd_hg, fd_hg_last, fd_nblk, fd_nr, fd_H, fd_P, fd_kus;
+  FastDiv fd_qpk;  // query heads per K/V head (H / H_kv)
 };
 
 // Number of keys u in [0, n_kv) of shard s that are visible to a query at global position

@@ -69,7 +69,7 @@ struct FmhaCfg {
   static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * STAGES);
   static constexpr int NBAR = 3 + 3 * STAGES + 9 * 2;
   static constexpr int STATS_BYTES = 2 * 128 * 8;
-  static constexpr int PLAN_BYTES = 2 * 48;
+  static constexpr int PLAN_BYTES = 2 * 56;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES + PLAN_BYTES;
   static constexpr int THREADS = 512;
   static constexpr int D = DP;
@@ -238,6 +238,7 @@ __device__ __forceinline__ int item_of_cta(int k) {
 
 struct Item {
   int b, h, r, t0;
+  int hk;  // K/V head of query head h
   int rows_valid[2];
   long long pos0;      // global position of local query token 0 of shard r
   long long pos_last;  // position of the item's last valid query row
@@ -251,7 +252,7 @@ struct ItemPlan {
   int n;  // K/V tiles the item walks
   int pad;
 };
-static_assert(sizeof(ItemPlan) == 48, "plan slot size");
+static_assert(sizeof(ItemPlan) == 56, "plan slot size");
 
 // Items come in head groups of w.hgroup (batch, head) pairs, so the K/V the concurrently running
 // CTAs read stays in L2; inside a group the order is longest first with heads innermost.
@@ -279,6 +280,7 @@ __device__ __forceinline__ void decode_item(const AttnWork& w, int idx, Item& it
   }
   it.b = fdiv(bh, w.fd_H);
   it.h = bh - it.b * w.H;
+  it.hk = fdiv(it.h, w.fd_qpk);
   it.r = w.r_first + ri * w.r_step;
   it.t0 = blk * 256;
   it.rows_valid[0] = max(0, min(128, w.n_q - it.t0));
@@ -634,12 +636,12 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int cb = 0; cb < C::NCB; ++cb)
             tma_load_5d(sK + st * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_k, bar_k_full + st, cb * C::CB, wk.u0,
-                        wk.s, it.h, it.b);
+                        wk.s, it.hk, it.b);
           mbar_arrive_expect_tx(bar_v_full + st, C::TILE_BYTES);
 #pragma unroll
           for (int cb = 0; cb < C::NCB; ++cb)
             tma_load_5d(sV + st * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_v, bar_v_full + st, cb * C::CB, wk.u0,
-                        wk.s, it.h, it.b);
+                        wk.s, it.hk, it.b);
           ++g;
         }
       }

@@ -39,6 +39,7 @@ class Workload:
     qk_sigma: float = 1.0
     v_dist: str = "normal"  # "normal" (sigma 1) | "uniform" (U(-1, 1))
     tabular: tuple | None = None  # (batch, rows, features, embed, heads) for the row-axis layout
+    H_kv: int | None = None  # K/V heads (grouped-query attention); None = H
 
     @property
     def seed(self) -> int:
@@ -115,9 +116,10 @@ def make_qkv(w: Workload, seed: int | None = None, N: int | None = None):
                                     (n * feats * embed, hd, feats * embed, 1)))
         return tuple(out)
     shape = (w.B, w.H, n, w.d)
+    kv_shape = (w.B, w.H if w.H_kv is None else w.H_kv, n, w.d)
     q = draw(shape, seed, 0, "normal", w.qk_sigma, w.dtype)
-    k = draw(shape, seed, 1, "normal", w.qk_sigma, w.dtype)
-    v = draw(shape, seed, 2, w.v_dist, 1.0, w.dtype)
+    k = draw(kv_shape, seed, 1, "normal", w.qk_sigma, w.dtype)
+    v = draw(kv_shape, seed, 2, w.v_dist, 1.0, w.dtype)
     return q, k, v
 
 

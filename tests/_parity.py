@@ -26,6 +26,7 @@ def oracle_heads(q, k, v, scale, causal, pos_q=None, pos_k=None, rows=None):
     """Oracle O, LSE for every (b, h) of [B, H, N, d] host arrays; optionally only ``rows``."""
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
+    H_kv = k.shape[1]  # K/V heads (grouped-query attention when fewer than H)
     pos_q = np.arange(Nq) if pos_q is None else np.asarray(pos_q)
     pos_k = np.arange(Nk) if pos_k is None else np.asarray(pos_k)
     sel = np.arange(Nq) if rows is None else np.asarray(rows)
@@ -33,7 +34,8 @@ def oracle_heads(q, k, v, scale, causal, pos_q=None, pos_k=None, rows=None):
     lse = np.zeros((B, H, len(sel)))
     for b in range(B):
         for h in range(H):
-            o[b, h], lse[b, h] = oracle.attention_rows(q[b, h][sel], k[b, h], v[b, h], scale, pos_q[sel], pos_k,
+            hk = oracle.kv_head(h, H, H_kv)
+            o[b, h], lse[b, h] = oracle.attention_rows(q[b, h][sel], k[b, hk], v[b, hk], scale, pos_q[sel], pos_k,
                                                         causal)
     return o, lse
 

@@ -64,7 +64,19 @@ def test_host_validation_without_a_device(ra):
     tq, tk = ra.tensor_desc(q), ra.tensor_desc(k)
     st = lib.ra_attn_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tk), ctypes.byref(tq), None,
                          ctypes.c_float(0.0), 0, None)
-    assert st == ra.RA_ERR_INVALID_ARG and b"B and H" in lib.ra_last_error()
+    assert st == ra.RA_ERR_INVALID_ARG and b"H_kv must divide" in lib.ra_last_error()
+    # grouped-query K/V: H_kv must divide H, and k, v must agree on it; B must agree
+    q4 = torch.zeros(1, 4, 16, 64, dtype=torch.bfloat16)
+    k2 = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)
+    v1 = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
+    kb = torch.zeros(2, 2, 16, 64, dtype=torch.bfloat16)
+    tq4, tk2, tv1, tkb = (ra.tensor_desc(x) for x in (q4, k2, v1, kb))
+    st = lib.ra_attn_fwd(ctypes.byref(tq4), ctypes.byref(tk2), ctypes.byref(tv1), ctypes.byref(tq4), None,
+                         ctypes.c_float(0.0), 0, None)
+    assert st == ra.RA_ERR_INVALID_ARG and b"same number of heads" in lib.ra_last_error()
+    st = lib.ra_attn_fwd(ctypes.byref(tq4), ctypes.byref(tkb), ctypes.byref(tkb), ctypes.byref(tq4), None,
+                         ctypes.c_float(0.0), 0, None)
+    assert st == ra.RA_ERR_INVALID_ARG and b"agree on B" in lib.ra_last_error()
     # bf16 head dim must be a multiple of 8 and <= 128
     q2 = torch.zeros(1, 1, 16, 136, dtype=torch.bfloat16)
     t2 = ra.tensor_desc(q2)

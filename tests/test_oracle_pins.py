@@ -458,6 +458,51 @@ def _typo_merge(o_a, lse_a, o_b, lse_b):
     return wa[..., None] * o_a + wb[..., None] * o_b, lse
 
 
+def check_kv_head(fn):
+    """Grouped-query head mapping as [VR] "MQA与GQA" fixes it: its 32Q/8KV figure puts query heads
+    1-4 on K/V head 1, 5-8 on K/V head 2, 9-12 on K/V head 3 (1-based there); as many groups as
+    heads is multi-head attention and one group is multi-query attention."""
+    try:
+        if [fn(h, 32, 8) for h in range(12)] != [0, 0, 0, 0, 1, 1, 1, 1, 2, 2, 2, 2]:
+            return False
+        if fn(31, 32, 8) != 7:
+            return False
+        if [fn(h, 8, 8) for h in range(8)] != [0, 1, 2, 3, 4, 5, 6, 7]:
+            return False
+        if [fn(h, 8, 1) for h in range(8)] != [0, 0, 0, 0, 0, 0, 0, 0]:
+            return False
+        return True
+    except Exception:
+        return False
+
+
+def test_kv_head_follows_the_pages_grouping():
+    assert check_kv_head(oracle.kv_head)
+    with pytest.raises(ValueError):
+        oracle.kv_head(0, 8, 3)  # K/V heads must divide the query heads
+    with pytest.raises(ValueError):
+        oracle.kv_head(8, 8, 2)
+
+
+def test_grouped_query_attention_equals_multi_head_on_repeated_kv():
+    """Each query head of a group attends with the group's shared K/V pair: identical to
+    multi-head attention whose K/V heads are copies of the shared pair."""
+    H, H_kv, n, d = 6, 2, 40, 8
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((H, n, d))
+    k = rng.standard_normal((H_kv, n, d))
+    v = rng.standard_normal((H_kv, n, d))
+    k_rep, v_rep = np.repeat(k, H // H_kv, axis=0), np.repeat(v, H // H_kv, axis=0)
+    pos = np.arange(n)
+    for causal in (False, True):
+        allowed = A.allowed_mask(pos, pos, causal) if causal else None
+        for h in range(H):
+            hk = oracle.kv_head(h, H, H_kv)
+            o_g, l_g = oracle.attention(q[h], k[hk], v[hk], 0.35, allowed)
+            o_m, l_m = oracle.attention(q[h], k_rep[h], v_rep[h], 0.35, allowed)
+            assert np.array_equal(o_g, o_m) and np.array_equal(l_g, l_m)
+
+
 @pytest.mark.parametrize("name,check", [
     ("lse sign typo", lambda: check_lse_pair(_typo_lse_pair)),
     ("merge built on the typo", lambda: check_worked_merge(_typo_merge)),
@@ -468,6 +513,8 @@ def _typo_merge(o_a, lse_a, o_b, lse_b):
     ("online softmax without O rescale", lambda: check_worked_attention(
         lambda q, k, v, s, al: _unrescaled_online(q, k, v, s, al, block=1))),
     ("split merge without weights", lambda: check_split_merge(A.attention, _unnormalised_merge)),
+    ("query heads interleaved over K/V heads", lambda: check_kv_head(lambda h, n, g: h % g)),
+    ("group size taken as the number of K/V heads", lambda: check_kv_head(lambda h, n, g: h // g)),
 ])
 def test_planted_mistakes_are_caught(name, check):
     with np.errstate(all="ignore"):
@@ -476,6 +523,7 @@ def test_planted_mistakes_are_caught(name, check):
 
 def test_pins_pass_on_the_oracle():
     assert check_lse_pair(oracle.lse_pair)
+    assert check_kv_head(oracle.kv_head)
     assert check_worked_merge(oracle.merge_pair)
     assert check_worked_attention(oracle.attention)
     assert check_split_merge(oracle.attention, oracle.merge_pair)
