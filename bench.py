@@ -240,8 +240,14 @@ class OracleSampler:
         hk = oracle.kv_head(h, w.H, self.k.shape[1])  # K/V head (grouped-query K/V)
         k = self.k[b, hk].astype(np.float64)
         v = self.v[b, hk].astype(np.float64)
-        oracle.attention_rows(self.q[b, h][rows].astype(np.float64), k, v, w.scale, rows, pos, w.causal)
-        keys = (rows + 1).sum() if w.causal else self.rows * w.N
+        oracle.attention_rows(self.q[b, h][rows].astype(np.float64), k, v, w.scale, rows, pos, w.causal,
+                              window=w.window)
+        if w.window is not None:
+            keys = np.minimum(rows + 1, w.window).sum()
+        elif w.causal:
+            keys = (rows + 1).sum()
+        else:
+            keys = self.rows * w.N
         self.flops += 4.0 * w.d * float(keys)
 
 
@@ -291,8 +297,10 @@ def run_reference(args, w):
 # ---------------------------------------------------------------------------------------------
 def config_dict(w, args):
     name = w.name if w.H_kv is None else f"{w.name}, grouped-query K/V with {w.H_kv} heads"
+    if w.window is not None:
+        name += f", sliding window of {w.window} positions"
     return {"workload": f"cfg{w.cfg}: {name}", "B": w.B, "H": w.H, "H_kv": w.H_kv or w.H, "N": w.N, "d": w.d,
-            "causal": w.causal,
+            "causal": w.causal, "window": w.window,
             "P": w.P, "layout": w.layout, "schedule": args.schedule,
             "l2": "flushed between timed steps (256 MiB write outside the events)",
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
@@ -322,7 +330,7 @@ def run_gpu(args, w):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        ra.ring_fwd(q, k, v, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws)
+        ra.ring_fwd(q, k, v, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws, w.window or 0)
 
     launches_per_step = 1 if (args.schedule == "fused" or w.P == 1) else w.P
 
@@ -362,7 +370,7 @@ def run_gpu(args, w):
     def e2e_step():
         for dst, src in zip((qd, kd, vd), (qp, kp, vp)):
             dst.copy_(src, non_blocking=True)
-        ra.ring_fwd(qd, kd, vd, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws)
+        ra.ring_fwd(qd, kd, vd, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws, w.window or 0)
         o_host.copy_(o, non_blocking=True)
         lse_host.copy_(lse, non_blocking=True)
 
@@ -412,7 +420,7 @@ def run_gpu(args, w):
     if rank != 0:
         return 0
     peak = peaks["bf16_tflops"]
-    traffic_key = f"cfg{w.cfg}" if w.H_kv is None else f"cfg{w.cfg}-kv{w.H_kv}"
+    traffic_key = f"cfg{w.cfg}" + ("" if w.H_kv is None else f"-kv{w.H_kv}") + ("" if w.window is None else f"-w{w.window}")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -424,7 +432,8 @@ def run_gpu(args, w):
                      "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s", "frac": (value / world) / peak,
                      "traffic": args.traffic if args.traffic is not None else recorded_traffic(traffic_key,
                                                                                                   args.schedule),
-                     "note": "algorithmic FLOPs (4*B*H*N^2*d, halved when causal) / summed duration of the step's "
+                     "note": "algorithmic FLOPs (4*d per visible query-key pair: 4*B*H*N^2*d, halved when causal; "
+                             "sum_i min(i+1, w) pairs per head with a sliding window w) / summed duration of the step's "
                              f"{launches_per_step} serialised launches (CUDA events on the launch stream)"},
         "mufu_roofline": mufu_roofline(w, ms, world, clocks.summary()),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -455,6 +464,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-merge", action="store_true")
+    ap.add_argument("--window", type=int, default=None,
+                    help="causal sliding-window variant of a causal workload (window in positions)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query variant of the workload: K and V with this many heads (must divide H)")
     ap.add_argument("--traffic", type=float, default=None,
@@ -471,6 +482,12 @@ def main(argv=None):
         import dataclasses
 
         w = dataclasses.replace(w, H_kv=args.kv_heads)
+    if args.window is not None:
+        if not w.causal or args.window < 1:
+            raise SystemExit("--window needs a causal workload and a window >= 1")
+        import dataclasses
+
+        w = dataclasses.replace(w, window=args.window)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

@@ -102,13 +102,23 @@ typedef struct {
 } ra_pos_t;
 
 /* Single full pass (ring with P = 1).
- * q [B,H,Nq,d]; k, v [B,H,Nk,d] (or [B,H_kv,Nk,d], see above); o [B,H,Nq,d] with o->dtype == q->dtype (bf16 in -> bf16 out,
- * fp32 in -> fp32 out); lse: fp32 [B,H,Nq] contiguous, may be NULL.  scale <= 0 selects
+ * q [B,H,Nq,d]; k, v [B,H,Nk,d] (or [B,H_kv,Nk,d], see above); o [B,H,Nq,d] with
+ * o->dtype == q->dtype (bf16 in -> bf16 out, fp32 in -> fp32 out); lse: fp32 [B,H,Nq] contiguous, may be NULL.  scale <= 0 selects
  * 1/sqrt(d).  causal != 0: query i and key j both sit at position = index (0-based), key j is
  * visible iff j <= i.  o must not overlap q, k or v. */
 ra_status_t ra_attn_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
                         const ra_tensor_t* o, float* lse, float scale, int causal,
                         ra_stream_t stream);
+
+/* Sliding-window attention (vibe-research page, "Sliding Window Attention": each token attends
+ * only to the w most recent tokens; only the mask changes).  As ra_attn_fwd with causal = 1, and
+ * key j is visible to query i iff i - window < j <= i: the window's most recent positions, the
+ * query's own included (window = 1: each token attends to itself only; window >= Nk: plain
+ * causal).  window < 1 returns RA_ERR_INVALID_ARG.  (Extension beyond the calls the pages' ring
+ * method needs.) */
+ra_status_t ra_attn_fwd_window(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
+                               const ra_tensor_t* o, float* lse, float scale, int64_t window,
+                               ra_stream_t stream);
 
 /* One ring step: the partial attention of a query shard against one KV shard.
  * k_shard, v_shard hold the shard's keys/values (any strided view, e.g. every P-th row of the
@@ -168,6 +178,14 @@ ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
                         int layout, int causal, float scale, int schedule,
                         const ra_tensor_t* o, float* lse, const ra_stream_t* streams,
                         int n_streams, void* workspace, size_t workspace_bytes);
+
+/* ra_ring_fwd with a causal sliding window of `window` positions (as ra_attn_fwd_window, on
+ * global token positions, either layout, either schedule).  window < 1 returns
+ * RA_ERR_INVALID_ARG.  Shard pairs and key tiles wholly outside every row's window are skipped. */
+ra_status_t ra_ring_fwd_window(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P,
+                               int layout, int64_t window, float scale, int schedule,
+                               const ra_tensor_t* o, float* lse, const ra_stream_t* streams,
+                               int n_streams, void* workspace, size_t workspace_bytes);
 
 /* ra_ring_fwd with the RA_RING_STEPWISE schedule for callers that cannot allocate device memory
  * at the point of the call: code recording a CUDA graph (cudaMalloc cannot be captured), code

@@ -53,13 +53,24 @@ def token_positions(layout: str, P: int, shard: int, n_local: int) -> np.ndarray
     raise ValueError(f"unknown layout {layout!r}")
 
 
-def allowed_mask(pos_q: np.ndarray, pos_k: np.ndarray, causal: bool) -> np.ndarray:
-    """Boolean [Nq, Nk]: may query i attend key j?  Causal iff pos_k <= pos_q."""
+def allowed_mask(pos_q: np.ndarray, pos_k: np.ndarray, causal: bool, window=None) -> np.ndarray:
+    """Boolean [Nq, Nk]: may query i attend key j?  Causal iff pos_k <= pos_q.
+
+    ``window`` (causal only): a sliding window of that many positions, [VR] "Sliding Window
+    Attention" (each token attends only to the w most recent tokens): additionally
+    pos_k > pos_q - window, so the query's own position and the window - 1 before it."""
     pos_q = np.asarray(pos_q, dtype=np.int64)
     pos_k = np.asarray(pos_k, dtype=np.int64)
     if not causal:
+        if window is not None:
+            raise ValueError("a sliding window is defined for causal attention only")
         return np.ones((pos_q.shape[0], pos_k.shape[0]), dtype=bool)
-    return pos_k[None, :] <= pos_q[:, None]
+    allowed = pos_k[None, :] <= pos_q[:, None]
+    if window is not None:
+        if window < 1:
+            raise ValueError("window must be >= 1")
+        allowed &= pos_k[None, :] > pos_q[:, None] - window
+    return allowed
 
 
 def _masked_scores(q, k, scale, allowed):
@@ -107,7 +118,7 @@ def attention(q, k, v, scale: float, allowed=None):
     return o, lse
 
 
-def attention_rows(q_rows, k, v, scale: float, pos_q, pos_k, causal: bool, chunk: int = 64):
+def attention_rows(q_rows, k, v, scale: float, pos_q, pos_k, causal: bool, chunk: int = 64, window=None):
     """``attention`` for a subset of query rows (given with their global positions).
 
     Used to check large problems on sampled rows; rows are processed ``chunk`` at
@@ -119,7 +130,7 @@ def attention_rows(q_rows, k, v, scale: float, pos_q, pos_k, causal: bool, chunk
     lse = np.zeros(q_rows.shape[0])
     for a in range(0, q_rows.shape[0], chunk):
         b = min(a + chunk, q_rows.shape[0])
-        allowed = allowed_mask(pos_q[a:b], pos_k, causal) if causal else None
+        allowed = allowed_mask(pos_q[a:b], pos_k, causal, window) if causal else None
         o[a:b], lse[a:b] = attention(q_rows[a:b], k, v, scale, allowed)
     return o, lse
 

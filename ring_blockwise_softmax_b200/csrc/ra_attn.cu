@@ -416,14 +416,16 @@ ra_status_t set_last_error(ra_status_t status, const char* message) { return fai
 // ==============================================================================================
 extern "C" {
 
-ra_status_t ra_attn_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, const ra_tensor_t* o,
-                        float* lse, float scale, int causal, ra_stream_t stream) {
+static ra_status_t attn_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
+                                 const ra_tensor_t* o, float* lse, float scale, int causal, int64_t window,
+                                 ra_stream_t stream) {
   ra_status_t st = check_qkv(q, k, v);
   if (st != RA_OK) return st;
   if ((st = check_out(o, q, "o", q->dtype)) != RA_OK) return st;
   DevInfo dev;
   if ((st = current_device(&dev)) != RA_OK) return st;
   ra::AttnWork w = base_work(q, scale, causal, dev);
+  w.window = window;
   w.n_q = static_cast<int>(q->shape[2]);
   w.n_kv = static_cast<int>(k->shape[2]);
   w.n_q_tiles = (w.n_q + q_rows_per_cta(q->dtype) - 1) / q_rows_per_cta(q->dtype);
@@ -598,9 +600,10 @@ ra_status_t ra_ring_workspace_size(const ra_tensor_t* q, int P, int schedule, si
   return ok();
 }
 
-ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P, int layout,
-                        int causal, float scale, int schedule, const ra_tensor_t* o, float* lse,
-                        const ra_stream_t* streams, int n_streams, void* workspace, size_t workspace_bytes) {
+static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P,
+                                 int layout, int causal, int64_t window, float scale, int schedule,
+                                 const ra_tensor_t* o, float* lse, const ra_stream_t* streams, int n_streams,
+                                 void* workspace, size_t workspace_bytes) {
   ra_status_t st = check_qkv(q, k, v);
   if (st != RA_OK) return st;
   if ((st = check_out(o, q, "o", q->dtype)) != RA_OK) return st;
@@ -628,6 +631,7 @@ ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
   const int64_t tok_rows = striped ? P : 1;
 
   ra::AttnWork w = base_work(q, scale, causal, dev);
+  w.window = window;
   w.P = P;
   w.n_q = static_cast<int>(n_local);
   w.n_kv = static_cast<int>(n_local);
@@ -721,6 +725,32 @@ ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
     if (e != cudaSuccess) return cuda_fail(e, "stream join");
   }
   return st == RA_OK ? ok() : st;
+}
+
+ra_status_t ra_attn_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, const ra_tensor_t* o,
+                        float* lse, float scale, int causal, ra_stream_t stream) {
+  return attn_fwd_impl(q, k, v, o, lse, scale, causal, 0, stream);
+}
+
+ra_status_t ra_attn_fwd_window(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
+                               const ra_tensor_t* o, float* lse, float scale, int64_t window, ra_stream_t stream) {
+  if (window < 1) return fail(RA_ERR_INVALID_ARG, "window must be >= 1 (got %lld)", (long long)window);
+  return attn_fwd_impl(q, k, v, o, lse, scale, 1, window, stream);
+}
+
+ra_status_t ra_ring_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P, int layout,
+                        int causal, float scale, int schedule, const ra_tensor_t* o, float* lse,
+                        const ra_stream_t* streams, int n_streams, void* workspace, size_t workspace_bytes) {
+  return ring_fwd_impl(q, k, v, P, layout, causal, 0, scale, schedule, o, lse, streams, n_streams, workspace,
+                       workspace_bytes);
+}
+
+ra_status_t ra_ring_fwd_window(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P, int layout,
+                               int64_t window, float scale, int schedule, const ra_tensor_t* o, float* lse,
+                               const ra_stream_t* streams, int n_streams, void* workspace, size_t workspace_bytes) {
+  if (window < 1) return fail(RA_ERR_INVALID_ARG, "window must be >= 1 (got %lld)", (long long)window);
+  return ring_fwd_impl(q, k, v, P, layout, 1, window, scale, schedule, o, lse, streams, n_streams, workspace,
+                       workspace_bytes);
 }
 
 ra_status_t ra_get_device_status(ra_stream_t stream) {

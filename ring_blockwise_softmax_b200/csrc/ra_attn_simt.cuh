@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(128)
   const long long q_pos0 = w.q_off + static_cast<long long>(r) * w.q_rstep;
   const long long pos_q = q_pos0 + static_cast<long long>(tq) * w.q_tstride;
   const long long pos_last = q_pos0 + static_cast<long long>(tile * kSimtRows + rows_valid - 1) * w.q_tstride;
+  const long long pos_first = q_pos0 + static_cast<long long>(tile * kSimtRows) * w.q_tstride;
 
   const float* qg = static_cast<const float*>(w.q);
   const float* kg = static_cast<const float*>(w.k);
@@ -61,8 +62,10 @@ __global__ void __launch_bounds__(128)
     int s = (r - (w.ring_step + step)) % w.P;
     if (s < 0) s += w.P;
     const int kv_lim = visible_key_limit(w, pos_last, s);
+    const int kv_start = visible_key_start(w, pos_first, s);  // keys before it: outside every row's window
     const int row_lim = row_ok ? visible_key_limit(w, pos_q, s) : 0;
-    for (int u0 = 0; u0 < kv_lim; u0 += kSimtKeys) {
+    const int row_lo = row_ok ? visible_key_start(w, pos_q, s) : 0;
+    for (int u0 = kv_start - kv_start % kSimtKeys; u0 < kv_lim; u0 += kSimtKeys) {
       __syncthreads();
       for (int e = threadIdx.x; e < kSimtKeys * DP; e += blockDim.x) {
         const int kr = e / DP, c = e % DP;
@@ -80,7 +83,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
         for (int i = 0; i < DH; ++i) part = fmaf(qv[i], sk[kr][half * DH + i], part);
         const float full = part + __shfl_xor_sync(0xffffffffu, part, 1);
-        const float x = (u0 + kr < row_lim) ? full * w.scale : -INFINITY;
+        const float x = (u0 + kr < row_lim && u0 + kr >= row_lo) ? full * w.scale : -INFINITY;
         sc[kr] = x;
         mt = fmaxf(mt, x);
       }

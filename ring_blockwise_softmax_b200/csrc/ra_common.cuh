@@ -354,6 +354,7 @@ struct AttnWork {
   int r_first, r_step, n_r;
   int ring_step;  // t
   int causal;
+  long long window;  // sliding window (causal only): keys at positions > pos_q - window; 0 = none
   long long q_off, q_rstep, q_tstride;
   long long k_off, k_sstep, k_ustride;
   float scale;       // softmax scale applied to q.k
@@ -403,6 +404,27 @@ __host__ __device__ __forceinline__ int visible_key_limit(const AttnWork& w, lon
   else
     quot = diff / stride;
   return quot < static_cast<unsigned long long>(w.n_kv) ? static_cast<int>(quot) + 1 : w.n_kv;
+}
+
+// First key u of shard s inside the sliding window of a query at global position pos_q: the keys
+// at positions pos_q - window + 1 ... pos_q (the window's most recent positions, the query's own
+// included; vibe-research page, "Sliding Window Attention": each token attends to the w most
+// recent tokens).  0 without a window.  (k_ustride >= 1.)
+__host__ __device__ __forceinline__ int visible_key_start(const AttnWork& w, long long pos_q, int s) {
+  if (w.window <= 0) return 0;
+  const long long base = w.k_off + static_cast<long long>(s) * w.k_sstep;
+  const long long first = pos_q - w.window + 1;  // first visible position
+  if (first <= base) return 0;
+  const unsigned long long diff = static_cast<unsigned long long>(first - base);  // > 0
+  const unsigned long long stride = static_cast<unsigned long long>(w.k_ustride);
+  unsigned long long quot;  // ceil(diff / stride)
+  if (stride == 1)
+    quot = diff;
+  else if (((diff + stride - 1) >> 31) == 0 && stride == w.fd_kus.d)
+    quot = static_cast<unsigned long long>(fdiv(static_cast<int>(diff + stride - 1), w.fd_kus));
+  else
+    quot = (diff + stride - 1) / stride;
+  return quot < static_cast<unsigned long long>(w.n_kv) ? static_cast<int>(quot) : w.n_kv;
 }
 
 // (r - t) mod P for 0 <= r < P, 0 <= t < 2P (the launch keeps ring_step + steps <= 2P).

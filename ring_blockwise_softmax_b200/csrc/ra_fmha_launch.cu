@@ -9,11 +9,11 @@
 
 namespace ra {
 
-template <int EPI>
+template <int EPI, bool WIN>
 static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
                               int n_steps, int sms, cudaStream_t stream) {
   using C = FmhaCfg<RA_FMHA_DP>;
-  auto kern = fmha_fwd_sm100<RA_FMHA_DP, EPI>;
+  auto kern = fmha_fwd_sm100<RA_FMHA_DP, EPI, WIN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // Persistent grid: one CTA per SM (at most one per work item of 256 query rows).
@@ -30,15 +30,21 @@ static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, cons
 cudaError_t RA_CAT(launch_fmha_dp, RA_FMHA_DP)(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                                const AttnWork& w, int n_steps, int epi, int sms,
                                                cudaStream_t stream) {
+  // Launches with a sliding window use their own instantiation (WIN = true).
+  const bool win = w.window > 0;
   switch (epi) {
     case kEpiOut:
-      return launch_epi<kEpiOut>(mq, mk, mv, w, n_steps, sms, stream);
+      return win ? launch_epi<kEpiOut, true>(mq, mk, mv, w, n_steps, sms, stream)
+                 : launch_epi<kEpiOut, false>(mq, mk, mv, w, n_steps, sms, stream);
     case kEpiPart:
-      return launch_epi<kEpiPart>(mq, mk, mv, w, n_steps, sms, stream);
+      return win ? launch_epi<kEpiPart, true>(mq, mk, mv, w, n_steps, sms, stream)
+                 : launch_epi<kEpiPart, false>(mq, mk, mv, w, n_steps, sms, stream);
     case kEpiAcc:
-      return launch_epi<kEpiAcc>(mq, mk, mv, w, n_steps, sms, stream);
+      return win ? launch_epi<kEpiAcc, true>(mq, mk, mv, w, n_steps, sms, stream)
+                 : launch_epi<kEpiAcc, false>(mq, mk, mv, w, n_steps, sms, stream);
     case kEpiAccOut:
-      return launch_epi<kEpiAccOut>(mq, mk, mv, w, n_steps, sms, stream);
+      return win ? launch_epi<kEpiAccOut, true>(mq, mk, mv, w, n_steps, sms, stream)
+                 : launch_epi<kEpiAccOut, false>(mq, mk, mv, w, n_steps, sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

@@ -69,7 +69,7 @@ struct FmhaCfg {
   static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * STAGES);
   static constexpr int NBAR = 3 + 3 * STAGES + 9 * 2;
   static constexpr int STATS_BYTES = 2 * 128 * 8;
-  static constexpr int PLAN_BYTES = 2 * 56;
+  static constexpr int PLAN_BYTES = 2 * 64;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES + PLAN_BYTES;
   static constexpr int THREADS = 512;
   static constexpr int D = DP;
@@ -240,8 +240,9 @@ struct Item {
   int b, h, r, t0;
   int hk;  // K/V head of query head h
   int rows_valid[2];
-  long long pos0;      // global position of local query token 0 of shard r
-  long long pos_last;  // position of the item's last valid query row
+  long long pos0;       // global position of local query token 0 of shard r
+  long long pos_last;   // position of the item's last valid query row
+  long long pos_first;  // position of the item's first query row
 };
 
 // A work item as the TMA producer publishes it to the other roles (decoded once per CTA).  Used
@@ -252,7 +253,7 @@ struct ItemPlan {
   int n;  // K/V tiles the item walks
   int pad;
 };
-static_assert(sizeof(ItemPlan) == 56, "plan slot size");
+static_assert(sizeof(ItemPlan) == 64, "plan slot size");
 
 // Items come in head groups of w.hgroup (batch, head) pairs, so the K/V the concurrently running
 // CTAs read stays in L2; inside a group the order is longest first with heads innermost.
@@ -288,6 +289,7 @@ __device__ __forceinline__ void decode_item(const AttnWork& w, int idx, Item& it
   it.pos0 = w.q_off + static_cast<long long>(it.r) * w.q_rstep;
   const int last = it.t0 + it.rows_valid[0] + it.rows_valid[1] - 1;
   it.pos_last = it.pos0 + static_cast<long long>(last) * w.q_tstride;
+  it.pos_first = it.pos0 + static_cast<long long>(it.t0) * w.q_tstride;
 }
 
 struct Walk {
@@ -297,39 +299,50 @@ struct Walk {
   int lim;   // keys of shard s visible to the item's last row
 };
 
+// Keys [start, lim) of shard s are visible to some row of the item: lim from its last row (the
+// causal bound), start from its first row (the sliding-window bound; 0 without a window).  The
+// walk covers the 128-key tiles that meet that range.  WIN: the launch has a sliding window
+// (compiled separately so that the plain path carries none of its arithmetic).
+template <bool WIN>
 __device__ __forceinline__ bool walk_seek(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
   for (; k.step < n_steps; ++k.step) {
     const int s = ring_shard(w, it.r, w.ring_step + k.step);
     const int lim = visible_key_limit(w, it.pos_last, s);
-    if (lim > 0) {
+    const int start = WIN ? visible_key_start(w, it.pos_first, s) : 0;
+    if (lim > start) {
       k.s = s;
       k.lim = lim;
-      k.u0 = 0;
+      k.u0 = start & ~(FmhaCfg<32>::BN - 1);
       return true;
     }
   }
   return false;
 }
 
+template <bool WIN>
 __device__ __forceinline__ bool walk_begin(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
   k.step = 0;
-  return walk_seek(k, w, it, n_steps);
+  return walk_seek<WIN>(k, w, it, n_steps);
 }
 
+template <bool WIN>
 __device__ __forceinline__ bool walk_next(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
   k.u0 += FmhaCfg<32>::BN;
   if (k.u0 < k.lim) return true;
   ++k.step;
-  return walk_seek(k, w, it, n_steps);
+  return walk_seek<WIN>(k, w, it, n_steps);
 }
 
 
 // Number of K/V tiles the item walks (what the MMA issuer needs; it never reads the keys).
+template <bool WIN>
 __device__ __forceinline__ int walk_count(const AttnWork& w, const Item& it, int n_steps) {
   int n = 0;
   for (int step = 0; step < n_steps; ++step) {
     const int s = ring_shard(w, it.r, w.ring_step + step);
-    n += (visible_key_limit(w, it.pos_last, s) + FmhaCfg<32>::BN - 1) / FmhaCfg<32>::BN;
+    const int lim = visible_key_limit(w, it.pos_last, s);
+    const int start = WIN ? visible_key_start(w, it.pos_first, s) : 0;
+    if (lim > start) n += (lim + FmhaCfg<32>::BN - 1) / FmhaCfg<32>::BN - start / FmhaCfg<32>::BN;
   }
   return n;
 }
@@ -516,7 +529,7 @@ __device__ __forceinline__ void softmax_exp_store(const uint32_t (&sr)[4][32], f
 // ---------------------------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------------------------
-template <int DP, int EPI>
+template <int DP, int EPI, bool WIN>
 __global__ void __launch_bounds__(512, 1)
     fmha_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnWork w, int n_steps, int n_items) {
@@ -609,12 +622,12 @@ __global__ void __launch_bounds__(512, 1)
           const int slot = it_seq & 1;
           if (it_seq >= 2 && !mbar_wait(bar_plan_empty + slot, ((it_seq >> 1) - 1) & 1, ctl, 0x103)) break;
           plan[slot].it = it;
-          plan[slot].n = walk_count(w, it, n_steps);
+          plan[slot].n = walk_count<WIN>(w, it, n_steps);
           mbar_arrive(bar_plan_full + slot);
           ++it_seq;
         }
         Walk wk;
-        bool has = walk_begin(wk, w, it, n_steps);
+        bool has = walk_begin<WIN>(wk, w, it, n_steps);
         if (!has) continue;
         if (it_q > 0 && !mbar_wait(bar_q_empty, (it_q - 1) & 1, ctl, 0x101)) break;
         mbar_arrive_expect_tx(bar_q_full, 2 * C::TILE_BYTES);
@@ -625,7 +638,7 @@ __global__ void __launch_bounds__(512, 1)
             tma_load_5d(sQ + q * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_q, bar_q_full, cb * C::CB,
                         it.t0 + 128 * q, it.r, it.h, it.b);
         ++it_q;
-        for (; has; has = walk_next(wk, w, it, n_steps)) {
+        for (; has; has = walk_next<WIN>(wk, w, it, n_steps)) {
           const int st = static_cast<int>(g % C::STAGES);
           if (g >= C::STAGES &&
               !mbar_wait(bar_kv_empty + st, static_cast<uint32_t>((g / C::STAGES) - 1) & 1, ctl, 0x102)) {
@@ -672,7 +685,7 @@ __global__ void __launch_bounds__(512, 1)
         if (idx >= n_items) continue;
         Item it;
         decode_item(w, idx, it);
-        const int n = walk_count(w, it, n_steps);
+        const int n = walk_count<WIN>(w, it, n_steps);
         if (n == 0) {
           for (int q = 0; q < 2 && ok && it_all > 0; ++q)
             ok = mbar_wait_issuer(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x208);
@@ -842,11 +855,12 @@ __global__ void __launch_bounds__(512, 1)
       float m_used = -INFINITY;  // running max of scaled scores, log2 units
       float l_sum = 0.f;         // running sum of 2^(x - m_used)
       Walk wk;
-      int cur_s = -1, row_lim = 0;
-      for (bool has = walk_begin(wk, w, it, n_steps); has; has = walk_next(wk, w, it, n_steps)) {
+      int cur_s = -1, row_lim = 0, row_lo = 0;
+      for (bool has = walk_begin<WIN>(wk, w, it, n_steps); has; has = walk_next<WIN>(wk, w, it, n_steps)) {
         if (wk.s != cur_s) {
           cur_s = wk.s;
           row_lim = row_ok ? visible_key_limit(w, pos_q, wk.s) : w.n_kv;
+          if (WIN) row_lo = row_ok ? visible_key_start(w, pos_q, wk.s) : 0;
         }
         if (!__all_sync(0xffffffffu, s_seen)) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + q, c & 1, ctl, 0x301));
@@ -866,12 +880,14 @@ __global__ void __launch_bounds__(512, 1)
           tc_fence_before();
           mbar_arrive(bar_s_free + q);
         }
-        const int lim = row_lim - wk.u0;  // keys [0, lim) of this tile are visible to this row
-        const bool masked = __any_sync(0xffffffffu, lim < C::BN);
-        if (lim < C::BN) {
+        const int lim = row_lim - wk.u0;  // keys [lo, lim) of this tile are visible to this row
+        const int lo = WIN ? row_lo - wk.u0 : 0;
+        const bool cut = WIN ? (lim < C::BN || lo > 0) : lim < C::BN;
+        const bool masked = __any_sync(0xffffffffu, cut);
+        if (cut) {
 #pragma unroll
           for (int e = 0; e < 128; ++e)
-            if (e >= lim) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
+            if (e >= lim || (WIN && e < lo)) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
         }
         // Row max as 8 independent chains (a single chain of 128 dependent max operations would
         // be latency-bound).
@@ -989,7 +1005,7 @@ __global__ void __launch_bounds__(512, 1)
       } else {
         decode_item(w, idx, it);
         Walk wk;
-        has_o = walk_begin(wk, w, it, n_steps);
+        has_o = walk_begin<WIN>(wk, w, it, n_steps);
       }
       for (int q = 0; q < 2; ++q) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_full + q, it_all & 1, ctl, 0x401) &&

@@ -40,6 +40,7 @@ class Workload:
     v_dist: str = "normal"  # "normal" (sigma 1) | "uniform" (U(-1, 1))
     tabular: tuple | None = None  # (batch, rows, features, embed, heads) for the row-axis layout
     H_kv: int | None = None  # K/V heads (grouped-query attention); None = H
+    window: int | None = None  # causal sliding window (positions); None = none
 
     @property
     def seed(self) -> int:
@@ -50,7 +51,12 @@ class Workload:
         return 1.0 / math.sqrt(self.d)
 
     def flops(self) -> float:
-        """Algorithmic forward FLOPs: 4*B*H*N^2*d, halved when causal."""
+        """Algorithmic forward FLOPs: 4*B*H*N^2*d, halved when causal; with a sliding window of w
+        positions, 4*B*H*d per visible pair, sum_i min(i + 1, w) pairs per head."""
+        if self.window is not None:
+            w, n = self.window, self.N
+            pairs = w * (w + 1) / 2 + (n - w) * w if w < n else n * (n + 1) / 2
+            return 4.0 * self.B * self.H * self.d * pairs
         f = 4.0 * self.B * self.H * self.N * self.N * self.d
         return f / 2 if self.causal else f
 

@@ -41,8 +41,8 @@ SCHEDULES = {"stepwise": RA_RING_STEPWISE, "fused": RA_RING_FUSED}
 
 # Exported symbols of the library, in header order (the CPU test checks each one is present).
 SYMBOLS = (
-    "ra_attn_fwd", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_workspace_size",
-    "ra_ring_fwd", "ra_ring_fwd_noalloc", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
+    "ra_attn_fwd", "ra_attn_fwd_window", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_workspace_size",
+    "ra_ring_fwd", "ra_ring_fwd_window", "ra_ring_fwd_noalloc", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
     "ra_debug_exp2", "ra_status_string", "ra_last_error", "ra_version",
 )
 
@@ -61,6 +61,7 @@ _F = ctypes.c_void_p  # float* (device)
 _S = ctypes.c_void_p  # cudaStream_t
 
 _lib.ra_attn_fwd.argtypes = [_T, _T, _T, _T, _F, ctypes.c_float, ctypes.c_int, _S]
+_lib.ra_attn_fwd_window.argtypes = [_T, _T, _T, _T, _F, ctypes.c_float, ctypes.c_int64, _S]
 _lib.ra_attn_partial.argtypes = [_T, _T, _T, RaPos, RaPos, ctypes.c_int, ctypes.c_float, _T, _F, ctypes.c_int, _S]
 _lib.ra_lse_merge.argtypes = [_F, _F, _F, _F, _F, _F, ctypes.c_int64, ctypes.c_int, _S]
 _lib.ra_lse_merge_n.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, _F,
@@ -68,6 +69,9 @@ _lib.ra_lse_merge_n.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(
 _lib.ra_ring_workspace_size.argtypes = [_T, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
 _lib.ra_ring_fwd.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int, _T,
                              _F, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t]
+_lib.ra_ring_fwd_window.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_int,
+                                    _T, _F, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_void_p,
+                                    ctypes.c_size_t]
 _lib.ra_ring_fwd_noalloc.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, _T, _F,
                                      _S]
 _lib.ra_get_device_status.argtypes = [_S]
@@ -154,9 +158,14 @@ def _stream(stream):
 # entry points (same names as the C ABI, without the ra_ prefix)
 # ---------------------------------------------------------------------------------------------
 
-def attn_fwd(q, k, v, o, lse=None, scale: float = 0.0, causal: bool = False, stream=None):
-    """ra_attn_fwd: O (and LSE, natural log) of softmax(scale*QK^T)V into the given buffers."""
+def attn_fwd(q, k, v, o, lse=None, scale: float = 0.0, causal: bool = False, stream=None, window: int = 0):
+    """ra_attn_fwd: O (and LSE, natural log) of softmax(scale*QK^T)V into the given buffers.
+    window > 0: ra_attn_fwd_window (causal sliding window of that many positions)."""
     tq, tk, tv, to = (tensor_desc(x) for x in (q, k, v, o))
+    if window:
+        _check(_lib.ra_attn_fwd_window(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(to),
+                                       _ptr(lse), float(scale), int(window), _stream(stream)), "ra_attn_fwd_window")
+        return
     _check(_lib.ra_attn_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(to), _ptr(lse),
                             float(scale), int(bool(causal)), _stream(stream)), "ra_attn_fwd")
 
@@ -197,8 +206,9 @@ def ring_workspace_size(q, P: int, schedule: str = "stepwise") -> int:
 
 
 def ring_fwd(q, k, v, P: int, layout: str, causal: bool, o, lse=None, scale: float = 0.0,
-             schedule: str = "stepwise", streams=None, workspace=None):
-    """ra_ring_fwd: ring attention over P virtual shards (contiguous or striped) on one GPU."""
+             schedule: str = "stepwise", streams=None, workspace=None, window: int = 0):
+    """ra_ring_fwd: ring attention over P virtual shards (contiguous or striped) on one GPU.
+    window > 0: ra_ring_fwd_window (causal sliding window of that many positions)."""
     import torch
 
     if streams is None:
@@ -207,6 +217,11 @@ def ring_fwd(q, k, v, P: int, layout: str, causal: bool, o, lse=None, scale: flo
     tq, tk, tv, to = (tensor_desc(x) for x in (q, k, v, o))
     ws_ptr = None if workspace is None else ctypes.c_void_p(workspace.data_ptr())
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if window:
+        _check(_lib.ra_ring_fwd_window(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), int(P), LAYOUTS[layout],
+                                       int(window), float(scale), SCHEDULES[schedule], ctypes.byref(to), _ptr(lse),
+                                       arr, len(streams), ws_ptr, ws_bytes), "ra_ring_fwd_window")
+        return
     _check(_lib.ra_ring_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), int(P), LAYOUTS[layout],
                             int(bool(causal)), float(scale), SCHEDULES[schedule], ctypes.byref(to), _ptr(lse), arr,
                             len(streams), ws_ptr, ws_bytes), "ra_ring_fwd")
@@ -245,20 +260,22 @@ def debug_exp2(x, y_poly=None, y_mufu=None, stream=None):
 # conveniences that allocate outputs with torch (device memory only; compute stays in the lib)
 # ---------------------------------------------------------------------------------------------
 
-def attention(q, k, v, causal: bool = False, scale: float = 0.0, stream=None):
-    """Allocate O (dtype of q) and fp32 LSE, run ra_attn_fwd, return (O, LSE)."""
+def attention(q, k, v, causal: bool = False, scale: float = 0.0, stream=None, window: int = 0):
+    """Allocate O (dtype of q) and fp32 LSE, run ra_attn_fwd (ra_attn_fwd_window when window > 0),
+    return (O, LSE)."""
     import torch
 
     B, H, N, d = q.shape
     o = torch.empty((B, H, N, d), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    attn_fwd(q, k, v, o, lse, scale, causal, stream)
+    attn_fwd(q, k, v, o, lse, scale, causal, stream, window)
     return o, lse
 
 
 def ring_attention(q, k, v, P: int, layout: str = "contiguous", causal: bool = False, scale: float = 0.0,
-                   schedule: str = "stepwise", streams=None):
-    """Allocate O, LSE and the workspace, run ra_ring_fwd, return (O, LSE)."""
+                   schedule: str = "stepwise", streams=None, window: int = 0):
+    """Allocate O, LSE and the workspace, run ra_ring_fwd (ra_ring_fwd_window when window > 0),
+    return (O, LSE)."""
     import torch
 
     B, H, N, d = q.shape
@@ -266,7 +283,7 @@ def ring_attention(q, k, v, P: int, layout: str = "contiguous", causal: bool = F
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     nbytes = ring_workspace_size(q, P, schedule)
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device) if nbytes > 0 else None
-    ring_fwd(q, k, v, P, layout, causal, o, lse, scale, schedule, streams, ws)
+    ring_fwd(q, k, v, P, layout, causal, o, lse, scale, schedule, streams, ws, window)
     return o, lse
 
 

@@ -22,7 +22,7 @@ def to64(t):
     return t.detach().to("cpu").double().numpy()
 
 
-def oracle_heads(q, k, v, scale, causal, pos_q=None, pos_k=None, rows=None):
+def oracle_heads(q, k, v, scale, causal, pos_q=None, pos_k=None, rows=None, window=None):
     """Oracle O, LSE for every (b, h) of [B, H, N, d] host arrays; optionally only ``rows``."""
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
@@ -36,7 +36,7 @@ def oracle_heads(q, k, v, scale, causal, pos_q=None, pos_k=None, rows=None):
         for h in range(H):
             hk = oracle.kv_head(h, H, H_kv)
             o[b, h], lse[b, h] = oracle.attention_rows(q[b, h][sel], k[b, hk], v[b, hk], scale, pos_q[sel], pos_k,
-                                                        causal)
+                                                        causal, window=window)
     return o, lse
 
 

@@ -77,6 +77,10 @@ def test_host_validation_without_a_device(ra):
     st = lib.ra_attn_fwd(ctypes.byref(tq4), ctypes.byref(tkb), ctypes.byref(tkb), ctypes.byref(tq4), None,
                          ctypes.c_float(0.0), 0, None)
     assert st == ra.RA_ERR_INVALID_ARG and b"agree on B" in lib.ra_last_error()
+    # a sliding window must cover at least the query's own position
+    st = lib.ra_attn_fwd_window(ctypes.byref(tq4), ctypes.byref(tq4), ctypes.byref(tq4), ctypes.byref(tq4), None,
+                                ctypes.c_float(0.0), 0, None)
+    assert st == ra.RA_ERR_INVALID_ARG and b"window" in lib.ra_last_error()
     # bf16 head dim must be a multiple of 8 and <= 128
     q2 = torch.zeros(1, 1, 16, 136, dtype=torch.bfloat16)
     t2 = ra.tensor_desc(q2)

@@ -503,6 +503,63 @@ def test_grouped_query_attention_equals_multi_head_on_repeated_kv():
             assert np.array_equal(o_g, o_m) and np.array_equal(l_g, l_m)
 
 
+def check_window_mask(mask_fn):
+    """Sliding window as [VR] "Sliding Window Attention" fixes it: each token attends only to the
+    w most recent tokens (its own included).  Six tokens, w = 3, written out by hand; w = 1 is the
+    identity; w >= N is plain causal; the allowed pairs number sum_i min(i + 1, w), the O(n w)
+    cost the section states (955 for n = 100, w = 10)."""
+    try:
+        pos = np.arange(6)
+        want = np.array([[1, 0, 0, 0, 0, 0],
+                         [1, 1, 0, 0, 0, 0],
+                         [1, 1, 1, 0, 0, 0],
+                         [0, 1, 1, 1, 0, 0],
+                         [0, 0, 1, 1, 1, 0],
+                         [0, 0, 0, 1, 1, 1]], dtype=bool)
+        if not np.array_equal(mask_fn(pos, pos, True, 3), want):
+            return False
+        if not np.array_equal(mask_fn(pos, pos, True, 1), np.eye(6, dtype=bool)):
+            return False
+        if not np.array_equal(mask_fn(pos, pos, True, 6), mask_fn(pos, pos, True, None)):
+            return False
+        if int(mask_fn(np.arange(100), np.arange(100), True, 10).sum()) != 955:
+            return False
+        return True
+    except Exception:
+        return False
+
+
+def test_sliding_window_mask():
+    assert check_window_mask(A.allowed_mask)
+    with pytest.raises(ValueError):
+        A.allowed_mask(np.arange(4), np.arange(4), False, 2)  # defined for causal attention only
+    with pytest.raises(ValueError):
+        A.allowed_mask(np.arange(4), np.arange(4), True, 0)
+
+
+def test_window_of_one_attends_to_itself():
+    """w = 1: every row's only key is its own, so O = v_i and LSE = s_ii exactly."""
+    n, d = 9, 5
+    q, k, v = _rand(n, d, 51), _rand(n, d, 52), _rand(n, d, 53)
+    pos = np.arange(n)
+    o, lse = oracle.attention(q, k, v, 0.4, A.allowed_mask(pos, pos, True, 1))
+    assert np.allclose(o, v, rtol=0, atol=1e-15)
+    assert np.allclose(lse, 0.4 * np.einsum("ij,ij->i", q, k), rtol=0, atol=1e-15)
+
+
+def _window_off_by_one(pos_q, pos_k, causal, window=None):
+    m = pos_k[None, :] <= pos_q[:, None]
+    if window is not None:
+        m &= pos_k[None, :] >= pos_q[:, None] - window
+    return m
+
+
+def _window_two_sided(pos_q, pos_k, causal, window=None):
+    if window is None:
+        return pos_k[None, :] <= pos_q[:, None]
+    return np.abs(pos_k[None, :] - pos_q[:, None]) < window
+
+
 @pytest.mark.parametrize("name,check", [
     ("lse sign typo", lambda: check_lse_pair(_typo_lse_pair)),
     ("merge built on the typo", lambda: check_worked_merge(_typo_merge)),
@@ -515,6 +572,8 @@ def test_grouped_query_attention_equals_multi_head_on_repeated_kv():
     ("split merge without weights", lambda: check_split_merge(A.attention, _unnormalised_merge)),
     ("query heads interleaved over K/V heads", lambda: check_kv_head(lambda h, n, g: h % g)),
     ("group size taken as the number of K/V heads", lambda: check_kv_head(lambda h, n, g: h // g)),
+    ("window one position too wide", lambda: check_window_mask(_window_off_by_one)),
+    ("window reaching into the future", lambda: check_window_mask(_window_two_sided)),
 ])
 def test_planted_mistakes_are_caught(name, check):
     with np.errstate(all="ignore"):
@@ -522,6 +581,7 @@ def test_planted_mistakes_are_caught(name, check):
 
 
 def test_pins_pass_on_the_oracle():
+    assert check_window_mask(A.allowed_mask)
     assert check_lse_pair(oracle.lse_pair)
     assert check_kv_head(oracle.kv_head)
     assert check_worked_merge(oracle.merge_pair)
