@@ -19,8 +19,9 @@ Sources (web pages, cited by title and section):
 * [KK]  git.kang-kang.com, "注意力机制演进": timeline (Striped Attention),
         "FlashAttention" data-flow figure, "Ring Attention" figure.
 * [FA]  intelliparadigm.com, "深度学习注意力机制优化与FlashAttention实践":
-        §2.1 (standard attention), §2.2 (memory arithmetic), §4.2 (online
-        softmax pseudocode), §5.1 (fp32 for log/exp, causal mask).
+        §2.1 (standard attention), §2.2 (memory arithmetic), §3.3 and §4.1
+        (the backward pass recomputes the weights), §4.2 (online softmax
+        pseudocode), §5.1 (fp32 for log/exp, causal mask).
 * [MO]  intelliparadigm.com, "Mosaic多轴注意力分片：突破Transformer长序列处理瓶颈":
         §2.1 (softmax(QK^T/sqrt(d))V, 150k-token memory), §2.2 (tabular
         tensors), §3.2 (ring steps: GPU 0 receives K3,V3 from GPU 3).
@@ -45,5 +46,6 @@ from .fp64 import (  # noqa: F401
     ring_attention,
     score_matrix_bytes,
     kv_head,
+    attention_backward,
 )
 from .sampling import sample_rows  # noqa: F401

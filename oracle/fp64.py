@@ -263,3 +263,28 @@ def kv_head(h: int, n_heads: int, n_kv_heads: int) -> int:
     if not 0 <= h < n_heads:
         raise ValueError("query head out of range")
     return h // (n_heads // n_kv_heads)
+
+
+def attention_backward(q, k, v, o, lse, do, scale: float, allowed=None):
+    """Gradients of one head's attention with respect to Q, K and V for the upstream gradient dO,
+    given the forward's saved O and LSE.  The attention weights are recomputed from LSE instead of
+    being stored ([FA] §3.3, §4.1 item 3: recompute the weights in the backward pass).  With
+    S = scale Q K^T, P = e^{S - LSE} on visible entries (0 elsewhere) and the chain rule through
+    the row softmax:
+      dV = P^T dO,   dP = dO V^T,   D_i = sum_c dO_ic O_ic,   dS = P * (dP - D),
+      dQ = scale dS K,   dK = scale dS^T Q.
+    Rows with LSE = -inf (no visible key) contribute nothing.  Returns (dQ, dK, dV) in float64."""
+    q, k, v, o, do = (np.asarray(x, np.float64) for x in (q, k, v, o, do))
+    lse = np.asarray(lse, np.float64)
+    s = _masked_scores(q, k, scale, allowed)
+    fin = np.isfinite(lse)
+    lse_safe = np.where(fin, lse, 0.0)
+    with np.errstate(invalid="ignore"):
+        p = np.where(fin[:, None] & np.isfinite(s), np.exp(s - lse_safe[:, None]), 0.0)
+    dv = p.T @ do
+    dp = do @ v.T
+    d_row = np.einsum("ic,ic->i", do, o)
+    ds = p * (dp - d_row[:, None])
+    dq = scale * (ds @ k)
+    dk = scale * (ds.T @ q)
+    return dq, dk, dv

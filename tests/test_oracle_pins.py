@@ -386,6 +386,88 @@ def test_against_torch_softmax_fp64():
         assert np.max(np.abs(l - want_l)) <= 1e-12
 
 
+def check_backward(bwd):
+    """The backward pass against an independent differentiation of the forward definition:
+    torch autograd in float64 through softmax(scale Q K^T + mask) V (non-causal, causal, and a
+    sliding window), and central finite differences of L = sum(dO * O) on a tiny case."""
+    try:
+        import torch
+    except ImportError:  # pragma: no cover
+        return True
+    for n, d, kind in ((40, 16, "full"), (37, 8, "causal"), (30, 12, "window")):
+        rng = np.random.default_rng(n * d)
+        q, k, v, do = (rng.normal(size=(n, d)) for _ in range(4))
+        scale = 0.7 / math.sqrt(d)
+        pos = np.arange(n)
+        allowed = None if kind == "full" else A.allowed_mask(pos, pos, True, 5 if kind == "window" else None)
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        sc = (tq @ tk.T) * scale
+        if allowed is not None:
+            sc = sc.masked_fill(torch.from_numpy(~allowed), float("-inf"))
+        (torch.softmax(sc, dim=-1) @ tv * torch.from_numpy(do)).sum().backward()
+        o, lse = oracle.attention(q, k, v, scale, allowed)
+        dq, dk, dv = bwd(q, k, v, o, lse, do, scale, allowed)
+        for got, want in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+            if np.asarray(got).shape != want.shape or np.max(np.abs(got - want.numpy())) > 1e-11:
+                return False
+    # finite differences: n = 4, d = 3
+    rng = np.random.default_rng(3)
+    q, k, v, do = (rng.normal(size=(4, 3)) for _ in range(4))
+    eps = 1e-6
+
+    def loss(q_, k_, v_):
+        o_, _ = oracle.attention(q_, k_, v_, 0.5)
+        return float((o_ * do).sum())
+
+    o, lse = oracle.attention(q, k, v, 0.5)
+    dq, dk, dv = bwd(q, k, v, o, lse, do, 0.5, None)
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        for idx in ((0, 0), (2, 1), (3, 2)):
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += eps
+            args_m[which][idx] -= eps
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            if abs(fd - grad[idx]) > 1e-7:
+                return False
+    return True
+
+
+def test_backward_against_autograd_and_finite_differences():
+    assert check_backward(oracle.attention_backward)
+
+
+def test_backward_row_without_visible_keys_is_zero():
+    """A query row with no visible key (LSE = -inf) passes no gradient anywhere."""
+    n, d = 6, 4
+    q, k, v, do = _rand(n, d, 61), _rand(n, d, 62), _rand(n, d, 63), _rand(n, d, 64)
+    allowed = np.ones((n, n), dtype=bool)
+    allowed[2] = False
+    o, lse = oracle.attention(q, k, v, 0.5, allowed)
+    assert np.isneginf(lse[2]) and np.all(o[2] == 0)
+    dq, dk, dv = oracle.attention_backward(q, k, v, o, lse, do, 0.5, allowed)
+    assert np.all(dq[2] == 0)
+    do2 = do.copy()
+    do2[2] = 0.0
+    _, dk2, dv2 = oracle.attention_backward(q, k, v, o, lse, do2, 0.5, allowed)
+    assert np.array_equal(dk, dk2) and np.array_equal(dv, dv2)
+
+
+def _bwd_without_d(q, k, v, o, lse, do, scale, allowed=None):
+    dq, dk, dv = A.attention_backward(q, k, v, np.zeros_like(np.asarray(o, float)), lse, do, scale, allowed)
+    return dq, dk, dv
+
+
+def _bwd_unscaled_dk(q, k, v, o, lse, do, scale, allowed=None):
+    dq, dk, dv = A.attention_backward(q, k, v, o, lse, do, scale, allowed)
+    return dq, dk / scale, dv
+
+
+def _bwd_dv_from_unnormalised_p(q, k, v, o, lse, do, scale, allowed=None):
+    dq, dk, dv = A.attention_backward(q, k, v, o, np.zeros_like(np.asarray(lse, float)), do, scale, allowed)
+    return dq, dk, dv
+
+
 # ---------------------------------------------------------------------------
 # 7. The pages' printed memory arithmetic
 # ---------------------------------------------------------------------------
@@ -574,6 +656,9 @@ def _window_two_sided(pos_q, pos_k, causal, window=None):
     ("group size taken as the number of K/V heads", lambda: check_kv_head(lambda h, n, g: h // g)),
     ("window one position too wide", lambda: check_window_mask(_window_off_by_one)),
     ("window reaching into the future", lambda: check_window_mask(_window_two_sided)),
+    ("backward without the row term D", lambda: check_backward(_bwd_without_d)),
+    ("backward dK missing the scale", lambda: check_backward(_bwd_unscaled_dk)),
+    ("backward weights not normalised by LSE", lambda: check_backward(_bwd_dv_from_unnormalised_p)),
 ])
 def test_planted_mistakes_are_caught(name, check):
     with np.errstate(all="ignore"):
@@ -581,6 +666,7 @@ def test_planted_mistakes_are_caught(name, check):
 
 
 def test_pins_pass_on_the_oracle():
+    assert check_backward(oracle.attention_backward)
     assert check_window_mask(A.allowed_mask)
     assert check_lse_pair(oracle.lse_pair)
     assert check_kv_head(oracle.kv_head)
