@@ -29,6 +29,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd TFLOP/s (bf16, ring P shards) and % of B200 dense BF16 peak"
+METRIC_BWD = "attention bwd TFLOP/s (recomputed weights, fp32 SIMT arithmetic) and % of B200 dense BF16 peak"
 SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -68,6 +69,16 @@ def mufu_roofline(w, ms: float, world: int, clocks: dict):
     peak = world * MUFU_EX2_PER_CLK_PER_SM * B200_SMS * mhz * 1e6 / 1e12
     return {"bound": "mufu", "achieved": achieved, "peak": peak, "unit": "Tex2/s", "frac": achieved / peak,
             "note": "one exponential per visible (query, key) pair; peak = 16 ex2/clk/SM x 148 SMs x sampled SM clock"}
+
+
+def fp32_roofline(achieved: float, clocks: dict):
+    """The backward kernels run their products as fp32 FMAs on the SIMT pipes: peak 128 FMA per
+    clock per SM (256 flops) x 148 SMs at the sampled SM clock."""
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    peak = 256 * B200_SMS * mhz * 1e6 / 1e12
+    return {"bound": "alu", "kernel": "attn_bwd_dq + attn_bwd_dkv", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "note": "10*d algorithmic flops per visible pair; peak = 128 fp32 FMA/clk/SM x 2 x 148 SMs x SM clock"}
 
 
 def recorded_traffic(workload: str, schedule: str):
@@ -333,6 +344,20 @@ def run_gpu(args, w):
         ra.ring_fwd(q, k, v, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws, w.window or 0)
 
     launches_per_step = 1 if (args.schedule == "fused" or w.P == 1) else w.P
+    if args.backward:
+        # Backward of the ring forward = backward on the full tensors (same function of global
+        # positions): ra_attn_bwd from the forward's saved O and LSE, dO drawn like the inputs.
+        step()
+        do_ = I.draw(tuple(q.shape), w.seed, 3, "normal", 1.0, w.dtype).to(dev)
+        dq_ = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        dk_ = torch.empty(k.shape, dtype=torch.float32, device=dev)
+        dv_ = torch.empty(v.shape, dtype=torch.float32, device=dev)
+        o_saved, lse_saved = o.clone(), lse.clone()
+
+        def step():  # noqa: F811 - the timed step of the backward mode
+            ra.attn_bwd(q, k, v, o_saved, lse_saved, do_, dq_, dk_, dv_, 0.0, w.causal, w.window or 0, stream)
+
+        launches_per_step = 2
 
     for _ in range(args.warmup):
         step()
@@ -355,7 +380,7 @@ def run_gpu(args, w):
     ms_local = sum(per_step_ms) / len(per_step_ms)
     ms = max_over_ranks(ms_local, world, dev)
     status = ra.get_device_status(stream)
-    flops = w.flops()
+    flops = w.flops() * (2.5 if args.backward else 1.0)  # backward: 5 products of 2*d per pair
     value = world * flops / (ms * 1e-3) / 1e12
 
     # End to end through the public API: pinned host inputs -> device, ring forward, result -> host.
@@ -373,6 +398,23 @@ def run_gpu(args, w):
         ra.ring_fwd(qd, kd, vd, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws, w.window or 0)
         o_host.copy_(o, non_blocking=True)
         lse_host.copy_(lse, non_blocking=True)
+
+    if args.backward:
+        # End to end for the backward: Q, K, V, O, LSE, dO in from pinned host memory, dQ, dK, dV out.
+        extra_in = [(x.to("cpu").pin_memory(), torch.empty_like(x)) for x in (o_saved, lse_saved, do_)]
+        grads_host = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in (dq_, dk_, dv_)]
+        h2d += sum(src.numel() * src.element_size() for src, _ in extra_in)
+        d2h = sum(g.numel() * g.element_size() for g in grads_host)
+
+        def e2e_step():  # noqa: F811 - the backward mode's end-to-end step
+            for dst, src in zip((qd, kd, vd), (qp, kp, vp)):
+                dst.copy_(src, non_blocking=True)
+            for src, dst in extra_in:
+                dst.copy_(src, non_blocking=True)
+            ra.attn_bwd(qd, kd, vd, extra_in[0][1], extra_in[1][1], extra_in[2][1], dq_, dk_, dv_, 0.0, w.causal,
+                        w.window or 0, stream)
+            for host, dev_t in zip(grads_host, (dq_, dk_, dv_)):
+                host.copy_(dev_t, non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -422,7 +464,8 @@ def run_gpu(args, w):
     peak = peaks["bf16_tflops"]
     traffic_key = f"cfg{w.cfg}" + ("" if w.H_kv is None else f"-kv{w.H_kv}") + ("" if w.window is None else f"-w{w.window}")
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if args.backward else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded, shapes and distributions of the workload)",
         "config": config_dict(w, args),
@@ -435,7 +478,8 @@ def run_gpu(args, w):
                      "note": "algorithmic FLOPs (4*d per visible query-key pair: 4*B*H*N^2*d, halved when causal; "
                              "sum_i min(i+1, w) pairs per head with a sliding window w) / summed duration of the step's "
                              f"{launches_per_step} serialised launches (CUDA events on the launch stream)"},
-        "mufu_roofline": mufu_roofline(w, ms, world, clocks.summary()),
+        "mufu_roofline": None if args.backward else mufu_roofline(w, ms, world, clocks.summary()),
+        "fp32_roofline": fp32_roofline(value / world, clocks.summary()) if args.backward else None,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
@@ -445,7 +489,7 @@ def run_gpu(args, w):
     }
     if merge is not None:
         line["merge"] = merge
-    if not args.skip_cpu and world == 1:
+    if not args.skip_cpu and world == 1 and not args.backward:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
     print(json.dumps(line), flush=True)
     return 0
@@ -464,6 +508,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-merge", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (ra_attn_bwd, fp32 SIMT kernels) instead of the forward")
     ap.add_argument("--window", type=int, default=None,
                     help="causal sliding-window variant of a causal workload (window in positions)")
     ap.add_argument("--kv-heads", type=int, default=None,

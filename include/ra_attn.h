@@ -157,6 +157,23 @@ ra_status_t ra_lse_merge_n(const float* const* o_parts, const float* const* lse_
 
 /* Workspace bytes ra_ring_fwd needs for (q, P, schedule): 0 for RA_RING_FUSED; for
  * RA_RING_STEPWISE an fp32 accumulator of B*H*N*(d+1)*4 bytes (plus alignment). */
+/* Backward pass (extension beyond the forward path the pages' ring method needs): gradients of
+ * L = sum(d_o * O) with respect to q, k, v for O = ra_attn_fwd(q, k, v, ..., scale, causal) (or
+ * ra_attn_fwd_window with window > 0), with the attention weights recomputed from the forward's
+ * saved lse instead of stored (intelliparadigm.com "深度学习注意力机制优化与FlashAttention实践",
+ * §3.3 and §4.1 item 3).  With P = e^{scale q k^T - lse} on visible entries:
+ *   dv = P^T d_o,  dS = P * (d_o v^T - rowsum(d_o * o)),  dq = scale dS k,  dk = scale dS^T q.
+ * q [B,H,Nq,d], k, v [B,H_kv,Nk,d] (grouped-query K/V: dk, dv sum over each group), o and d_o
+ * [B,H,Nq,d] of q's dtype (o the forward's output), lse fp32 [B,H,Nq] contiguous (the forward's),
+ * dq fp32 [B,H,Nq,d], dk, dv fp32 [B,H_kv,Nk,d]; all overwritten.  scale <= 0 selects 1/sqrt(d).
+ * window: 0, or with causal the forward's sliding window.  The backward of ra_ring_fwd (either
+ * layout or schedule) is this call on the same full tensors: the ring computes the same function
+ * of global positions.  Arithmetic is fp32 (SIMT kernels), inputs fp32 or bf16. */
+ra_status_t ra_attn_bwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
+                        const ra_tensor_t* o, const float* lse, const ra_tensor_t* d_o,
+                        const ra_tensor_t* dq, const ra_tensor_t* dk, const ra_tensor_t* dv,
+                        float scale, int causal, int64_t window, ra_stream_t stream);
+
 ra_status_t ra_ring_workspace_size(const ra_tensor_t* q, int P, int schedule, size_t* bytes);
 
 /* Ring attention over P virtual sequence shards on one GPU (vibe-research page, "Ring

@@ -17,6 +17,7 @@
 #include "ra_fmha_sm100.cuh"
 #include "ra_internal.h"
 #include "ra_lse_merge.cuh"
+#include "ra_attn_bwd.cuh"
 
 namespace ra {
 // Device status word: [0] OR of kDevStatus* flags, [1] site of the first wait that gave up.
@@ -751,6 +752,86 @@ ra_status_t ra_ring_fwd_window(const ra_tensor_t* q, const ra_tensor_t* k, const
   if (window < 1) return fail(RA_ERR_INVALID_ARG, "window must be >= 1 (got %lld)", (long long)window);
   return ring_fwd_impl(q, k, v, P, layout, 1, window, scale, schedule, o, lse, streams, n_streams, workspace,
                        workspace_bytes);
+}
+
+ra_status_t ra_attn_bwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, const ra_tensor_t* o,
+                        const float* lse, const ra_tensor_t* d_o, const ra_tensor_t* dq, const ra_tensor_t* dk,
+                        const ra_tensor_t* dv, float scale, int causal, int64_t window, ra_stream_t stream) {
+  ra_status_t st = check_qkv(q, k, v);
+  if (st != RA_OK) return st;
+  if ((st = check_tensor(o, "o")) != RA_OK) return st;
+  if ((st = check_tensor(d_o, "d_o")) != RA_OK) return st;
+  if ((st = check_tensor(dq, "dq")) != RA_OK) return st;
+  if ((st = check_tensor(dk, "dk")) != RA_OK) return st;
+  if ((st = check_tensor(dv, "dv")) != RA_OK) return st;
+  if (lse == nullptr) return fail(RA_ERR_INVALID_ARG, "lse is NULL (the forward's saved log-sum-exp is required)");
+  if (o->dtype != q->dtype || d_o->dtype != q->dtype) return fail(RA_ERR_INVALID_ARG, "o and d_o must have q's dtype");
+  if (dq->dtype != RA_F32 || dk->dtype != RA_F32 || dv->dtype != RA_F32)
+    return fail(RA_ERR_INVALID_ARG, "dq, dk, dv must be fp32");
+  for (int i = 0; i < 4; ++i) {
+    if (o->shape[i] != q->shape[i] || d_o->shape[i] != q->shape[i] || dq->shape[i] != q->shape[i])
+      return fail(RA_ERR_INVALID_ARG, "o, d_o and dq must have the shape of q");
+    if (dk->shape[i] != k->shape[i] || dv->shape[i] != k->shape[i])
+      return fail(RA_ERR_INVALID_ARG, "dk and dv must have the shape of k");
+  }
+  if (window < 0 || (window > 0 && !causal)) return fail(RA_ERR_INVALID_ARG, "window must be 0 or, with causal, >= 1");
+  DevInfo dev;
+  if ((st = current_device(&dev)) != RA_OK) return st;
+  ra::BwdWork w{};
+  w.B = static_cast<int>(q->shape[0]);
+  w.H = static_cast<int>(q->shape[1]);
+  w.H_kv = static_cast<int>(k->shape[1]);
+  w.n_q = static_cast<int>(q->shape[2]);
+  w.n_kv = static_cast<int>(k->shape[2]);
+  w.d = static_cast<int>(q->shape[3]);
+  w.causal = causal != 0;
+  w.window = window;
+  w.scale = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(w.d));
+  auto set = [](const ra_tensor_t* t, long long& sb, long long& sh, long long& st) {
+    sb = t->stride[0];
+    sh = t->stride[1];
+    st = t->stride[2];
+  };
+  w.q = q->data;
+  set(q, w.q_sb, w.q_sh, w.q_st);
+  w.k = k->data;
+  set(k, w.k_sb, w.k_sh, w.k_st);
+  w.v = v->data;
+  set(v, w.v_sb, w.v_sh, w.v_st);
+  w.o = o->data;
+  set(o, w.o_sb, w.o_sh, w.o_st);
+  w.d_o = d_o->data;
+  set(d_o, w.do_sb, w.do_sh, w.do_st);
+  w.lse = lse;
+  w.dq = static_cast<float*>(dq->data);
+  set(dq, w.dq_sb, w.dq_sh, w.dq_st);
+  w.dk = static_cast<float*>(dk->data);
+  set(dk, w.dk_sb, w.dk_sh, w.dk_st);
+  w.dv = static_cast<float*>(dv->data);
+  set(dv, w.dv_sb, w.dv_sh, w.dv_st);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int dp = padded_dim(w.d);
+  const dim3 gq((w.n_q + ra::kBwdRows - 1) / ra::kBwdRows, w.H, w.B);
+  const dim3 gk((w.n_kv + ra::kBwdRows - 1) / ra::kBwdRows, w.H_kv, w.B);
+  const unsigned threads = static_cast<unsigned>(ra::kBwdRows * (dp / ra::kBwdDH));
+#define RA_BWD_LAUNCH(T, DPV)                                  \
+  do {                                                         \
+    ra::attn_bwd_dq<T, DPV><<<gq, threads, 0, s>>>(w);         \
+    ra::attn_bwd_dkv<T, DPV><<<gk, threads, 0, s>>>(w);        \
+  } while (0)
+  if (q->dtype == RA_BF16) {
+    if (dp == 32) RA_BWD_LAUNCH(__nv_bfloat16, 32);
+    else if (dp == 64) RA_BWD_LAUNCH(__nv_bfloat16, 64);
+    else RA_BWD_LAUNCH(__nv_bfloat16, 128);
+  } else {
+    if (dp == 32) RA_BWD_LAUNCH(float, 32);
+    else if (dp == 64) RA_BWD_LAUNCH(float, 64);
+    else RA_BWD_LAUNCH(float, 128);
+  }
+#undef RA_BWD_LAUNCH
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+  return ok();
 }
 
 ra_status_t ra_get_device_status(ra_stream_t stream) {

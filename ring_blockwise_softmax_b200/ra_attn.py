@@ -41,7 +41,7 @@ SCHEDULES = {"stepwise": RA_RING_STEPWISE, "fused": RA_RING_FUSED}
 
 # Exported symbols of the library, in header order (the CPU test checks each one is present).
 SYMBOLS = (
-    "ra_attn_fwd", "ra_attn_fwd_window", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_workspace_size",
+    "ra_attn_fwd", "ra_attn_fwd_window", "ra_attn_bwd", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_workspace_size",
     "ra_ring_fwd", "ra_ring_fwd_window", "ra_ring_fwd_noalloc", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
     "ra_debug_exp2", "ra_status_string", "ra_last_error", "ra_version",
 )
@@ -62,6 +62,7 @@ _S = ctypes.c_void_p  # cudaStream_t
 
 _lib.ra_attn_fwd.argtypes = [_T, _T, _T, _T, _F, ctypes.c_float, ctypes.c_int, _S]
 _lib.ra_attn_fwd_window.argtypes = [_T, _T, _T, _T, _F, ctypes.c_float, ctypes.c_int64, _S]
+_lib.ra_attn_bwd.argtypes = [_T, _T, _T, _T, _F, _T, _T, _T, _T, ctypes.c_float, ctypes.c_int, ctypes.c_int64, _S]
 _lib.ra_attn_partial.argtypes = [_T, _T, _T, RaPos, RaPos, ctypes.c_int, ctypes.c_float, _T, _F, ctypes.c_int, _S]
 _lib.ra_lse_merge.argtypes = [_F, _F, _F, _F, _F, _F, ctypes.c_int64, ctypes.c_int, _S]
 _lib.ra_lse_merge_n.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, _F,
@@ -168,6 +169,26 @@ def attn_fwd(q, k, v, o, lse=None, scale: float = 0.0, causal: bool = False, str
         return
     _check(_lib.ra_attn_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(to), _ptr(lse),
                             float(scale), int(bool(causal)), _stream(stream)), "ra_attn_fwd")
+
+
+def attn_bwd(q, k, v, o, lse, d_o, dq, dk, dv, scale: float = 0.0, causal: bool = False, window: int = 0,
+             stream=None):
+    """ra_attn_bwd: fp32 dq, dk, dv of sum(d_o * O) from the forward's O and LSE (overwritten)."""
+    tq, tk, tv, to, tdo, tdq, tdk, tdv = (tensor_desc(x) for x in (q, k, v, o, d_o, dq, dk, dv))
+    _check(_lib.ra_attn_bwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(to), _ptr(lse),
+                            ctypes.byref(tdo), ctypes.byref(tdq), ctypes.byref(tdk), ctypes.byref(tdv), float(scale),
+                            int(bool(causal)), int(window), _stream(stream)), "ra_attn_bwd")
+
+
+def attention_backward(q, k, v, o, lse, d_o, causal: bool = False, scale: float = 0.0, window: int = 0, stream=None):
+    """Allocate fp32 dq, dk, dv, run ra_attn_bwd, return (dq, dk, dv)."""
+    import torch
+
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    attn_bwd(q, k, v, o, lse, d_o, dq, dk, dv, scale, causal, window, stream)
+    return dq, dk, dv
 
 
 def attn_partial(q, k_shard, v_shard, o_part, lse_part, q_pos=(0, 1), kv_pos=(0, 1), causal: bool = False,
