@@ -10,8 +10,9 @@
 // window of `window` positions.  K and V may have fewer heads than Q (grouped-query attention:
 // query head h uses K/V head h / (H / H_kv)); dK and dV then sum over the group.
 //
-// Two kernels, each over 64-row (or 64-key) blocks with DP / 32 threads per row, so a thread
-// holds 32 elements of each d-vector:
+// Two kernels, each over 64-row (or 64-key) blocks with TPR = DP / 32 threads per row, so a
+// thread holds 32 elements of each d-vector: thread p of a row owns elements p, p + TPR, ...,
+// which keeps the row's threads on different shared-memory banks:
 //   attn_bwd_dq  - a block of query rows walks the visible key tiles: dQ (and D, from dO and O);
 //   attn_bwd_dkv - a block of keys walks the query rows of every head of its group: dK, dV.
 // No atomics: every output element is owned by one thread.
@@ -88,13 +89,12 @@ __global__ void __launch_bounds__(kBwdRows * (DP / kBwdDH))
   const int row = threadIdx.x / TPR, part = threadIdx.x % TPR;
   const int i = blockIdx.x * kBwdRows + row;
   const bool row_ok = i < w.n_q;
-  const int c0 = part * kBwdDH;
 
   float qv[kBwdDH], dov[kBwdDH], acc[kBwdDH];
   float dsum = 0.f;
 #pragma unroll
   for (int e = 0; e < kBwdDH; ++e) {
-    const int c = c0 + e;
+    const int c = e * TPR + part;
     const bool in = row_ok && c < w.d;
     qv[e] = in ? ld_elem<T>(w.q, b * w.q_sb + h * w.q_sh + i * w.q_st + c) : 0.f;
     dov[e] = in ? ld_elem<T>(w.d_o, b * w.do_sb + h * w.do_sh + i * w.do_st + c) : 0.f;
@@ -125,13 +125,14 @@ __global__ void __launch_bounds__(kBwdRows * (DP / kBwdDH))
       sv[kr][c] = in ? ld_elem<T>(w.v, b * w.v_sb + hk * w.v_sh + j * w.v_st + c) : 0.f;
     }
     __syncthreads();
+#pragma unroll 4
     for (int kr = 0; kr < kBwdTile; ++kr) {
       const int j = j0 + kr;
       float s_part = 0.f, dp_part = 0.f;
 #pragma unroll
       for (int e = 0; e < kBwdDH; ++e) {
-        s_part = fmaf(qv[e], sk[kr][c0 + e], s_part);
-        dp_part = fmaf(dov[e], sv[kr][c0 + e], dp_part);
+        s_part = fmaf(qv[e], sk[kr][e * TPR + part], s_part);
+        dp_part = fmaf(dov[e], sv[kr][e * TPR + part], dp_part);
       }
       const float s = row_sum<TPR>(s_part) * w.scale;
       const float dp = row_sum<TPR>(dp_part);
@@ -139,13 +140,13 @@ __global__ void __launch_bounds__(kBwdRows * (DP / kBwdDH))
       const float p = vis ? expf(s - L) : 0.f;
       const float ds = p * (dp - D);
 #pragma unroll
-      for (int e = 0; e < kBwdDH; ++e) acc[e] = fmaf(ds, sk[kr][c0 + e], acc[e]);
+      for (int e = 0; e < kBwdDH; ++e) acc[e] = fmaf(ds, sk[kr][e * TPR + part], acc[e]);
     }
   }
   if (!row_ok) return;
 #pragma unroll
   for (int e = 0; e < kBwdDH; ++e) {
-    const int c = c0 + e;
+    const int c = e * TPR + part;
     if (c < w.d) w.dq[b * w.dq_sb + h * w.dq_sh + i * w.dq_st + c] = w.scale * acc[e];
   }
 }
@@ -163,12 +164,11 @@ __global__ void __launch_bounds__(kBwdRows * (DP / kBwdDH))
   const int key = threadIdx.x / TPR, part = threadIdx.x % TPR;
   const int j = blockIdx.x * kBwdRows + key;
   const bool key_ok = j < w.n_kv;
-  const int c0 = part * kBwdDH;
 
   float kv[kBwdDH], vv[kBwdDH], dk[kBwdDH], dv[kBwdDH];
 #pragma unroll
   for (int e = 0; e < kBwdDH; ++e) {
-    const int c = c0 + e;
+    const int c = e * TPR + part;
     const bool in = key_ok && c < w.d;
     kv[e] = in ? ld_elem<T>(w.k, b * w.k_sb + hk * w.k_sh + j * w.k_st + c) : 0.f;
     vv[e] = in ? ld_elem<T>(w.v, b * w.v_sb + hk * w.v_sh + j * w.v_st + c) : 0.f;
@@ -187,35 +187,39 @@ __global__ void __launch_bounds__(kBwdRows * (DP / kBwdDH))
   for (int g = 0; g < qpk; ++g) {
     const int h = hk * qpk + g;
     for (int i0 = i_begin; i0 < i_end; i0 += kBwdTile) {
+      // D_i = dO_i . O_i of the tile's rows, from O staged (coalesced) in the Q buffer.
       __syncthreads();
       for (int e = threadIdx.x; e < kBwdTile * DP; e += blockDim.x) {
         const int r = e / DP, c = e % DP;
         const int i = i0 + r;
         const bool in = i < w.n_q && c < w.d;
-        sq[r][c] = in ? ld_elem<T>(w.q, b * w.q_sb + h * w.q_sh + i * w.q_st + c) : 0.f;
+        sq[r][c] = in ? ld_elem<T>(w.o, b * w.o_sb + h * w.o_sh + i * w.o_st + c) : 0.f;
         sdo[r][c] = in ? ld_elem<T>(w.d_o, b * w.do_sb + h * w.do_sh + i * w.do_st + c) : 0.f;
       }
+      __syncthreads();
       if (threadIdx.x < kBwdTile) {
         const int r = threadIdx.x;
         const int i = i0 + r;
-        float dsum = 0.f, L = -INFINITY;
-        if (i < w.n_q) {
-          for (int c = 0; c < w.d; ++c)
-            dsum = fmaf(ld_elem<T>(w.d_o, b * w.do_sb + h * w.do_sh + i * w.do_st + c),
-                        ld_elem<T>(w.o, b * w.o_sb + h * w.o_sh + i * w.o_st + c), dsum);
-          L = w.lse[(static_cast<long long>(b) * w.H + h) * w.n_q + i];
-        }
+        float dsum = 0.f;
+        for (int c = 0; c < DP; ++c) dsum = fmaf(sdo[r][c], sq[r][c], dsum);
         s_d[r] = dsum;
-        s_lse[r] = L;
+        s_lse[r] = i < w.n_q ? w.lse[(static_cast<long long>(b) * w.H + h) * w.n_q + i] : -INFINITY;
       }
       __syncthreads();
+      for (int e = threadIdx.x; e < kBwdTile * DP; e += blockDim.x) {
+        const int r = e / DP, c = e % DP;
+        const int i = i0 + r;
+        sq[r][c] = (i < w.n_q && c < w.d) ? ld_elem<T>(w.q, b * w.q_sb + h * w.q_sh + i * w.q_st + c) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 4
       for (int r = 0; r < kBwdTile; ++r) {
         const int i = i0 + r;
         float s_part = 0.f, dp_part = 0.f;
 #pragma unroll
         for (int e = 0; e < kBwdDH; ++e) {
-          s_part = fmaf(sq[r][c0 + e], kv[e], s_part);
-          dp_part = fmaf(sdo[r][c0 + e], vv[e], dp_part);
+          s_part = fmaf(sq[r][e * TPR + part], kv[e], s_part);
+          dp_part = fmaf(sdo[r][e * TPR + part], vv[e], dp_part);
         }
         const float s = row_sum<TPR>(s_part) * w.scale;
         const float dp = row_sum<TPR>(dp_part);
@@ -225,8 +229,8 @@ __global__ void __launch_bounds__(kBwdRows * (DP / kBwdDH))
         const float ds = p * (dp - s_d[r]);
 #pragma unroll
         for (int e = 0; e < kBwdDH; ++e) {
-          dv[e] = fmaf(p, sdo[r][c0 + e], dv[e]);
-          dk[e] = fmaf(ds, sq[r][c0 + e], dk[e]);
+          dv[e] = fmaf(p, sdo[r][e * TPR + part], dv[e]);
+          dk[e] = fmaf(ds, sq[r][e * TPR + part], dk[e]);
         }
       }
     }
@@ -234,7 +238,7 @@ __global__ void __launch_bounds__(kBwdRows * (DP / kBwdDH))
   if (!key_ok) return;
 #pragma unroll
   for (int e = 0; e < kBwdDH; ++e) {
-    const int c = c0 + e;
+    const int c = e * TPR + part;
     if (c >= w.d) continue;
     w.dk[b * w.dk_sb + hk * w.dk_sh + j * w.dk_st + c] = w.scale * dk[e];
     w.dv[b * w.dv_sb + hk * w.dv_sh + j * w.dv_st + c] = dv[e];
