@@ -515,7 +515,7 @@ def main(argv=None):
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query variant of the workload: K and V with this many heads (must divide H)")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="DRAM bytes per launch of the attention kernel from an ncu capture of this build")
+                    help="DRAM bytes per launch of the attention kernel, from an ncu capture of the current kernel")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -56,7 +56,7 @@ typedef struct CUstream_st* ra_stream_t;
 typedef enum {
   RA_OK = 0,
   RA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, mismatched tensors, bad enum value */
-  RA_ERR_UNSUPPORTED = 2,  /* valid request this build cannot run (dtype, head dim, no sm_100) */
+  RA_ERR_UNSUPPORTED = 2,  /* valid request the library cannot run (dtype, head dim, no sm_100) */
   RA_ERR_ALIGNMENT = 3,    /* pointer or stride violates the 16-byte rule of the bf16 path */
   RA_ERR_WORKSPACE = 4,    /* ring workspace missing or smaller than ra_ring_workspace_size */
   RA_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed (message in ra_last_error) */

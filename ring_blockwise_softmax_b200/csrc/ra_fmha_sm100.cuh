@@ -228,8 +228,8 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 // ---------------------------------------------------------------------------------------------
 // Work items and the walk over KV tiles
 // ---------------------------------------------------------------------------------------------
-// Items are numbered longest first; CTA c takes item c in round 0, G-1-c in round 1, G+c in
-// round 2, ... (a snake over the G persistent CTAs), which pairs long with short items.
+// Items are numbered longest first; CTA c takes item c in its first sweep, G-1-c in its second,
+// G+c in its third, ... (a snake over the G persistent CTAs), which pairs long with short items.
 __device__ __forceinline__ int item_of_cta(int k) {
   const int G = static_cast<int>(gridDim.x);
   const int c = static_cast<int>(blockIdx.x);
