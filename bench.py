@@ -29,7 +29,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd TFLOP/s (bf16, ring P shards) and % of B200 dense BF16 peak"
-METRIC_BWD = "attention bwd TFLOP/s (recomputed weights, fp32 SIMT arithmetic) and % of B200 dense BF16 peak"
+METRIC_BWD = ("attention bwd TFLOP/s (weights recomputed from the saved LSE; bf16 inputs on the tensor cores) "
+              "and % of B200 dense BF16 peak")
 SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -71,8 +72,13 @@ def mufu_roofline(w, ms: float, world: int, clocks: dict):
             "note": "one exponential per visible (query, key) pair; peak = 16 ex2/clk/SM x 148 SMs x sampled SM clock"}
 
 
+BWD_NOTE = ("algorithmic FLOPs 10*d per visible query-key pair (S, dP, dV, dK, dQ products of 2*d each) / the "
+            "step's 2 serialised launches; the kernels execute 14*d (S and dP are recomputed by both the dQ and "
+            "the dK/dV instance)")
+
+
 def fp32_roofline(achieved: float, clocks: dict):
-    """The backward kernels run their products as fp32 FMAs on the SIMT pipes: peak 128 FMA per
+    """The fp32-input backward kernels run their products as fp32 FMAs on the SIMT pipes: peak 128 FMA per
     clock per SM (256 flops) x 148 SMs at the sampled SM clock."""
     mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
     peak = 256 * B200_SMS * mhz * 1e6 / 1e12
@@ -463,6 +469,8 @@ def run_gpu(args, w):
         return 0
     peak = peaks["bf16_tflops"]
     traffic_key = f"cfg{w.cfg}" + ("" if w.H_kv is None else f"-kv{w.H_kv}") + ("" if w.window is None else f"-w{w.window}")
+    if args.backward:
+        traffic_key += "-bwd"
     line = {
         "metric": METRIC_BWD if args.backward else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps,
@@ -471,15 +479,19 @@ def run_gpu(args, w):
         "config": config_dict(w, args),
         "pct_of_spec_bf16_peak": 100.0 * (value / world) / SPEC_BF16_TFLOPS,
         "pct_of_measured_bf16_peak": 100.0 * (value / world) / peak,
-        "roofline": {"bound": "tensor", "kernel": "fmha_fwd_sm100", "achieved": value / world, "peak": peak,
+        "roofline": {"bound": "tensor",
+                     "kernel": ("attn_bwd_sm100 (dQ + dK/dV instances)" if args.backward else "fmha_fwd_sm100"),
+                     "achieved": value / world, "peak": peak,
                      "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s", "frac": (value / world) / peak,
                      "traffic": args.traffic if args.traffic is not None else recorded_traffic(traffic_key,
                                                                                                   args.schedule),
-                     "note": "algorithmic FLOPs (4*d per visible query-key pair: 4*B*H*N^2*d, halved when causal; "
-                             "sum_i min(i+1, w) pairs per head with a sliding window w) / summed duration of the step's "
-                             f"{launches_per_step} serialised launches (CUDA events on the launch stream)"},
+                     "note": (BWD_NOTE if args.backward else
+                              "algorithmic FLOPs (4*d per visible query-key pair: 4*B*H*N^2*d, halved when causal; "
+                              "sum_i min(i+1, w) pairs per head with a sliding window w) / summed duration of the "
+                              f"step's {launches_per_step} serialised launches (CUDA events on the launch stream)")},
         "mufu_roofline": None if args.backward else mufu_roofline(w, ms, world, clocks.summary()),
-        "fp32_roofline": fp32_roofline(value / world, clocks.summary()) if args.backward else None,
+        "fp32_roofline": (fp32_roofline(value / world, clocks.summary())
+                          if args.backward and w.dtype == "f32" else None),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
@@ -509,7 +521,7 @@ def main(argv=None):
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-merge", action="store_true")
     ap.add_argument("--backward", action="store_true",
-                    help="time the backward pass (ra_attn_bwd, fp32 SIMT kernels) instead of the forward")
+                    help="time the backward pass (ra_attn_bwd) instead of the forward")
     ap.add_argument("--window", type=int, default=None,
                     help="causal sliding-window variant of a causal workload (window in positions)")
     ap.add_argument("--kv-heads", type=int, default=None,

@@ -3,7 +3,7 @@
     python -m ring_blockwise_softmax_b200.build [--force] [--verbose]
 
 Each translation unit is compiled in parallel into ``_build/`` (the tensor-core kernel once per
-padded head dim), then linked with the static CUDA runtime into a shared library next to this
+padded head dim, and so are the tensor-core backward kernels), then linked with the static CUDA runtime into a shared library next to this
 file.  Units are rebuilt only when a source or header is newer than their object.  The ptxas
 resource report (registers, spills, shared memory) of the last build is kept in
 ``_build/ptxas.log``.
@@ -36,6 +36,9 @@ UNITS = [
     ("ra_fmha_launch.cu", "fmha_dp32.o", ["-DRA_FMHA_DP=32"]),
     ("ra_fmha_launch.cu", "fmha_dp64.o", ["-DRA_FMHA_DP=64"]),
     ("ra_fmha_launch.cu", "fmha_dp128.o", ["-DRA_FMHA_DP=128"]),
+    ("ra_bwd_launch.cu", "bwd_dp32.o", ["-DRA_BWD_DP=32"]),
+    ("ra_bwd_launch.cu", "bwd_dp64.o", ["-DRA_BWD_DP=64"]),
+    ("ra_bwd_launch.cu", "bwd_dp128.o", ["-DRA_BWD_DP=128"]),
 ]
 
 

@@ -18,6 +18,7 @@
 #include "ra_internal.h"
 #include "ra_lse_merge.cuh"
 #include "ra_attn_bwd.cuh"
+#include "ra_bwd_sm100.cuh"
 
 namespace ra {
 // Device status word: [0] OR of kDevStatus* flags, [1] site of the first wait that gave up.
@@ -185,7 +186,7 @@ struct View5 {
   int64_t stride[5];  // stride[0] == 1
 };
 
-ra_status_t encode_view(CUtensorMap* map, const View5& v, int dp) {
+ra_status_t encode_view(CUtensorMap* map, const View5& v, int dp, int box_rows = 128) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   ra_status_t st = get_encode(&enc);
   if (st != RA_OK) return st;
@@ -199,7 +200,7 @@ ra_status_t encode_view(CUtensorMap* map, const View5& v, int dp) {
     strides[i - 1] = static_cast<cuuint64_t>(s) * 2;
   }
   const cuuint32_t box0 = dp == 32 ? 32 : 64;
-  cuuint32_t box[5] = {box0, 128, 1, 1, 1};
+  cuuint32_t box[5] = {box0, static_cast<cuuint32_t>(box_rows), 1, 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapSwizzle swz = dp == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(v.base), dims, strides, box, estr,
@@ -811,6 +812,61 @@ ra_status_t ra_attn_bwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
   set(dv, w.dv_sb, w.dv_sh, w.dv_st);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int dp = padded_dim(w.d);
+  if (q->dtype == RA_BF16 && w.H % w.H_kv == 0 && check_head_dim(w.d, RA_BF16) == RA_OK &&
+      check_tma_tensor(q, "q") == RA_OK && check_tma_tensor(k, "k") == RA_OK && check_tma_tensor(v, "v") == RA_OK &&
+      check_tma_tensor(o, "o") == RA_OK && check_tma_tensor(d_o, "d_o") == RA_OK) {
+    // Tensor-core path: dQ over blocks of 128 query rows, dK/dV over blocks of 128 keys.
+    ra::BwdMaps m;
+    struct {
+      CUtensorMap* map;
+      const ra_tensor_t* t;
+      int rows;
+    } maps[] = {{&m.q128, q, 128}, {&m.k128, k, 128}, {&m.v128, v, 128}, {&m.do128, d_o, 128}, {&m.q64, q, 64},
+                {&m.k64, k, 64},   {&m.v64, v, 64},   {&m.do64, d_o, 64}, {&m.o64, o, 64}};
+    for (auto& e : maps)
+      if ((st = encode_view(e.map, shard_view(e.t, e.t->shape[2], 1, 0, 1), dp, e.rows)) != RA_OK) return st;
+    ra::BwdTcWork tw{};
+    tw.B = w.B;
+    tw.H = w.H;
+    tw.H_kv = w.H_kv;
+    tw.n_q = w.n_q;
+    tw.n_kv = w.n_kv;
+    tw.d = w.d;
+    tw.qpk = w.H / w.H_kv;
+    tw.causal = w.causal;
+    tw.window = w.window;
+    tw.scale = w.scale;
+    tw.scale_log2 = static_cast<float>(w.scale * kLog2e);
+    tw.lse = lse;
+    tw.o = static_cast<const __nv_bfloat16*>(o->data);
+    tw.o_sb = w.o_sb;
+    tw.o_sh = w.o_sh;
+    tw.o_st = w.o_st;
+    tw.d_o = static_cast<const __nv_bfloat16*>(d_o->data);
+    tw.do_sb = w.do_sb;
+    tw.do_sh = w.do_sh;
+    tw.do_st = w.do_st;
+    tw.wait_limit_ns = g_wait_limit_ns.load();
+    tw.dev_status = dev.status;
+    ra::BwdTcWork wq = tw, wkv = tw;
+    wq.out1 = w.dq;
+    wq.o1_sb = w.dq_sb;
+    wq.o1_sh = w.dq_sh;
+    wq.o1_st = w.dq_st;
+    wkv.out1 = w.dk;
+    wkv.o1_sb = w.dk_sb;
+    wkv.o1_sh = w.dk_sh;
+    wkv.o1_st = w.dk_st;
+    wkv.out2 = w.dv;
+    wkv.o2_sb = w.dv_sb;
+    wkv.o2_sh = w.dv_sh;
+    wkv.o2_st = w.dv_st;
+    cudaError_t e = dp == 32 ? ra::launch_bwd_dp32(m, wq, wkv, s)
+                    : dp == 64 ? ra::launch_bwd_dp64(m, wq, wkv, s)
+                               : ra::launch_bwd_dp128(m, wq, wkv, s);
+    if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+    return ok();
+  }
   const dim3 gq((w.n_q + ra::kBwdRows - 1) / ra::kBwdRows, w.H, w.B);
   const dim3 gk((w.n_kv + ra::kBwdRows - 1) / ra::kBwdRows, w.H_kv, w.B);
   const unsigned threads = static_cast<unsigned>(ra::kBwdRows * (dp / ra::kBwdDH));

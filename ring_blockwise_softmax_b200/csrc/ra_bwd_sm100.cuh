@@ -1,0 +1,508 @@
+// ra_bwd_sm100.cuh - backward pass of softmax attention on the sm_100a tensor cores (bf16 inputs,
+// fp32 accumulation, fp32 gradients).
+//
+// What it computes: the gradients of L = sum(dO * O) with respect to Q, K and V for O =
+// softmax(scale Q K^T) V, with the attention weights recomputed from the forward's saved LSE
+// instead of being stored (intelliparadigm.com "深度学习注意力机制优化与FlashAttention实践" §3.3
+// and §4.1, item 3):
+//   P = e^{S - LSE} on visible entries (S = scale Q K^T),  D_i = sum_c dO_ic O_ic,
+//   dV = P^T dO,   dS = P * (dO V^T - D),   dQ = scale dS K,   dK = scale dS^T Q.
+// Visibility is the forward's: all keys, causal (key index <= query index), or a causal sliding
+// window of `window` positions; K and V may have fewer heads than Q (query head h uses K/V head
+// h / (H / H_kv)), and dK, dV then sum over the heads of the group.
+//
+// One kernel template serves both halves.  A CTA holds a FIXED block of 128 rows of two
+// operands (A1, A2) in shared memory and streams 64-row tiles of two or three others (B1, B2,
+// B3) through a STAGES-deep ring; per tile, with the fixed rows on the 128 tensor-memory lanes:
+//   S  = A1 B1^T,  dP = A2 B2^T             (tcgen05 SS form, fp32 in tensor memory)
+//   P  = exp2(S log2(e) - LSE log2(e)),  dS = P (dP - D)      (fp32 registers, stored as bf16
+//                                                             pairs into tensor memory)
+//   ACC1 += dS B1,  ACC2 += P B2            (TS form: A from tensor memory, B MN-major)
+// KV = true:  A1 = K, A2 = V of a block of keys, B1 = Q, B2 = dO, B3 = O of 64 query rows of
+//             every query head of the K/V head's group: ACC1 = dK / scale, ACC2 = dV.  The
+//             query rows' LSE and D (= dO . O, from the staged O tile) go through shared memory.
+// KV = false: A1 = Q, A2 = dO of a block of query rows, B1 = K, B2 = V of 64 keys:
+//             ACC1 = dQ / scale.  The rows' LSE and D sit in registers.
+// S and dP here are the transposes of each other's roles in the two instances, so both use the
+// forward's operand forms unchanged.  No atomics: every gradient element has one owner.
+//
+// Roles (320 threads): warps 0-7 element-wise (thread = tensor-memory lane (warp % 4) * 32 +
+// lane; warps 0-3 take columns 0-31 of a tile, warps 4-7 columns 32-63) and, at the end, the
+// epilogue; warp 8 TMA producer (and tensor-memory allocation); warp 9 MMA issuer.  The issuer
+// starts S, dP of tile j + 1 as soon as the element-wise warps hold those of tile j in
+// registers, so the tensor core works while they compute.  Every wait is bounded.
+#pragma once
+
+#include "ra_common.cuh"
+
+namespace ra {
+
+struct BwdTcWork {
+  int B, H, H_kv, n_q, n_kv, d;
+  int qpk;  // H / H_kv
+  int causal;
+  long long window;  // 0 = none (causal only)
+  float scale;
+  float scale_log2;  // scale * log2(e)
+  const float* lse;  // [B, H, n_q] contiguous (natural log)
+  // O and dO, read directly for the per-row D of the dQ instance.
+  const __nv_bfloat16* o;
+  long long o_sb, o_sh, o_st;
+  const __nv_bfloat16* d_o;
+  long long do_sb, do_sh, do_st;
+  // Outputs: out1 = dQ (KV = false) or dK (KV = true); out2 = dV (KV = true).  fp32.
+  float* out1;
+  long long o1_sb, o1_sh, o1_st;
+  float* out2;
+  long long o2_sb, o2_sh, o2_st;
+  unsigned long long wait_limit_ns;
+  unsigned int* dev_status;
+};
+
+template <int DP, bool KV>
+struct BwdCfg {
+  static_assert(DP == 32 || DP == 64 || DP == 128, "padded head dim must be 32, 64 or 128");
+  static constexpr int BM = 128;  // fixed rows (tensor-memory lanes)
+  static constexpr int BN = 64;   // rows of a streamed tile (tensor-memory columns of S, dP)
+  static constexpr int CB = (DP == 32) ? 32 : 64;  // columns per TMA box / swizzle span
+  static constexpr int NCB = DP / CB;
+  static constexpr int ROW_BYTES = CB * 2;
+  static constexpr uint32_t SWZ = (DP == 32) ? kSwizzle64B : kSwizzle128B;
+  static constexpr int ATOM_BYTES = 8 * ROW_BYTES;
+  static constexpr int BLK_M = BM * ROW_BYTES;  // one column block of a fixed operand
+  static constexpr int BLK_N = BN * ROW_BYTES;  // one column block of a streamed operand
+  static constexpr int FIX_BYTES = BM * DP * 2;
+  static constexpr int TILE_BYTES = BN * DP * 2;
+  static constexpr int NSTREAM = KV ? 3 : 2;
+  static constexpr int STAGE_BYTES = NSTREAM * TILE_BYTES;
+  static constexpr int STAGES_FIT = (192 * 1024 - 2 * FIX_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
+  static_assert(STAGES >= 2, "shared memory holds fewer than two stages");
+  static constexpr int NACC = KV ? 2 : 1;
+  // Tensor-memory columns (512 allocated): S, dP (fp32), P, dS (bf16 pairs), ACC1, ACC2.
+  static constexpr int S_COL = 0;
+  static constexpr int DP_COL = 64;
+  static constexpr int P_COL = 128;
+  static constexpr int DS_COL = 160;
+  static constexpr int ACC_COL = 256;
+  static_assert(ACC_COL + NACC * DP <= 512, "tensor memory overflow");
+  // Barriers: fixed_full, stage_full[S], stage_empty[S], s_full, s_free, p_full, pv_done,
+  // acc_done, stats_ready[2].
+  static constexpr int NBAR = 1 + 2 * STAGES + 5 + 2;
+  static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + NBAR * 8 + 16 + 4 * BN * 4;
+  static constexpr int THREADS = 320;
+};
+
+// The streamed tiles of one CTA: tiles tb .. te-1 (of BN rows) of each of `heads` streamed heads.
+struct BwdRange {
+  int b, hf;     // batch, head of the fixed operands
+  int m0;        // first fixed row
+  int tb, te;    // streamed tile range
+  int heads;     // streamed heads (query heads of the group, or 1)
+  int n;         // heads * (te - tb), or 0
+};
+
+template <bool KV>
+__device__ __forceinline__ BwdRange bwd_range(const BwdTcWork& w) {
+  BwdRange r;
+  r.b = blockIdx.z;
+  r.hf = blockIdx.y;
+  constexpr int BM = 128, BN = 64;
+  if (KV) {
+    // Key blocks in launch order: the first ones are seen by the most query rows (causal).
+    r.m0 = blockIdx.x * BM;
+    const int m_last = min(r.m0 + BM, w.n_kv) - 1;
+    const int lo = w.causal ? r.m0 : 0;
+    int hi = w.n_q;
+    if (w.causal && w.window > 0) hi = static_cast<int>(min(static_cast<long long>(w.n_q), m_last + w.window));
+    r.heads = w.qpk;
+    r.tb = lo / BN;
+    r.te = lo < hi ? (hi + BN - 1) / BN : r.tb;
+  } else {
+    // Query blocks last-first: under a causal mask the last rows see the most keys.
+    r.m0 = (gridDim.x - 1 - blockIdx.x) * BM;
+    const int m_last = min(r.m0 + BM, w.n_q) - 1;
+    const int hi = w.causal ? min(w.n_kv, m_last + 1) : w.n_kv;
+    int lo = 0;
+    if (w.causal && w.window > 0) lo = static_cast<int>(max(0LL, r.m0 - w.window + 1));
+    r.heads = 1;
+    r.tb = lo / BN;
+    r.te = lo < hi ? (hi + BN - 1) / BN : r.tb;
+  }
+  r.n = r.heads * (r.te - r.tb);
+  return r;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // low 16 bits = lo
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bwd_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Keep the compiler from using `r` before an earlier tcgen05.wait::ld (a second register array
+// loaded before the same wait).
+__device__ __forceinline__ void reg_pin32(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
+__device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, unsigned site) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctl, site));
+}
+
+__device__ __forceinline__ void bwd_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) break;
+  }
+}
+
+template <int DP, bool KV>
+__global__ void __launch_bounds__(320, 1)
+    attn_bwd_sm100(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
+                   const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
+                   const __grid_constant__ CUtensorMap tm_b3, const BwdTcWork w) {
+  using C = BwdCfg<DP, KV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sFix = smem;                        // A1 | A2
+  uint8_t* sStage = smem + 2 * C::FIX_BYTES;   // STAGES x (B1 | B2 [| B3])
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + C::STAGES * C::STAGE_BYTES);
+  uint64_t* bar_fixed = bars;
+  uint64_t* bar_stage_full = bars + 1;
+  uint64_t* bar_stage_empty = bar_stage_full + C::STAGES;
+  uint64_t* bar_s_full = bar_stage_empty + C::STAGES;
+  uint64_t* bar_s_free = bar_s_full + 1;
+  uint64_t* bar_p_full = bar_s_free + 1;
+  uint64_t* bar_pv_done = bar_p_full + 1;
+  uint64_t* bar_acc_done = bar_pv_done + 1;
+  uint64_t* bar_stats = bar_acc_done + 1;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_stats + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_lse2 = reinterpret_cast<float*>(tmem_slot + 4);  // [2][BN]  LSE log2(e) of streamed rows (KV)
+  float* s_dd = s_lse2 + 2 * C::BN;                          // [2][BN]  D of streamed rows (KV)
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  WaitCtl ctl{abort_flag, w.wait_limit_ns, w.dev_status};
+  const BwdRange rg = bwd_range<KV>(w);
+  const int nt = rg.te - rg.tb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_fixed, 1);
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(bar_stage_full + i, 1);
+      mbar_init(bar_stage_empty + i, KV ? 1 + 256 : 1);  // MMA commit (+ the D readers of O)
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_s_free, 256);
+    mbar_init(bar_p_full, 256);
+    mbar_init(bar_pv_done, 1);
+    mbar_init(bar_acc_done, 1);
+    mbar_init(bar_stats + 0, 256);
+    mbar_init(bar_stats + 1, 256);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    if (lane == 0) {
+      tma_prefetch_map(&tm_a1);
+      tma_prefetch_map(&tm_a2);
+      tma_prefetch_map(&tm_b1);
+      tma_prefetch_map(&tm_b2);
+      if (KV) tma_prefetch_map(&tm_b3);
+    }
+    __syncwarp();
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0 && rg.n > 0) {
+      // ================================================================ TMA producer
+      mbar_arrive_expect_tx(bar_fixed, 2 * C::FIX_BYTES);
+#pragma unroll
+      for (int cb = 0; cb < C::NCB; ++cb) {
+        tma_load_5d(sFix + cb * C::BLK_M, &tm_a1, bar_fixed, cb * C::CB, rg.m0, 0, rg.hf, rg.b);
+        tma_load_5d(sFix + C::FIX_BYTES + cb * C::BLK_M, &tm_a2, bar_fixed, cb * C::CB, rg.m0, 0, rg.hf, rg.b);
+      }
+      int g = 0, t = rg.tb, j = 0;
+      for (; j < rg.n; ++j) {
+        const int st = j % C::STAGES;
+        if (j >= C::STAGES && !mbar_wait(bar_stage_empty + st, ((j / C::STAGES) - 1) & 1, ctl, 0x701)) break;
+        const int hs = KV ? rg.hf * w.qpk + g : rg.hf / w.qpk;  // streamed head
+        uint8_t* dst = sStage + st * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(bar_stage_full + st, C::STAGE_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < C::NCB; ++cb) {
+          tma_load_5d(dst + cb * C::BLK_N, &tm_b1, bar_stage_full + st, cb * C::CB, t * C::BN, 0, hs, rg.b);
+          tma_load_5d(dst + C::TILE_BYTES + cb * C::BLK_N, &tm_b2, bar_stage_full + st, cb * C::CB, t * C::BN, 0,
+                      hs, rg.b);
+          if (KV)
+            tma_load_5d(dst + 2 * C::TILE_BYTES + cb * C::BLK_N, &tm_b3, bar_stage_full + st, cb * C::CB,
+                        t * C::BN, 0, hs, rg.b);
+        }
+        if (++t == rg.te) {
+          t = rg.tb;
+          ++g;
+        }
+      }
+      // No TMA write may still be in flight when the CTA exits.
+      bwd_drain(bar_fixed, 0, w.wait_limit_ns);
+      for (int i = (j > C::STAGES ? j - C::STAGES : 0); i < j; ++i)
+        bwd_drain(bar_stage_full + i % C::STAGES, (i / C::STAGES) & 1, w.wait_limit_ns);
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      // ================================================================ MMA issuer
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, C::BN, 0, 0);
+      constexpr uint32_t idesc_acc = make_idesc_bf16(128, DP, 0, 1);
+      const uint64_t kmaj = make_smem_desc(0, 16, C::ATOM_BYTES, C::SWZ);
+      const uint64_t mn = make_smem_desc(0, C::BLK_N, C::ATOM_BYTES, C::SWZ);
+      const uint32_t a1 = smem_addr(sFix), a2 = a1 + C::FIX_BYTES;
+      const uint32_t stage0 = smem_addr(sStage);
+      bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
+      for (int j = 0; ok && j <= rg.n; ++j) {
+        if (j < rg.n) {
+          const int st = j % C::STAGES;
+          if (!mbar_wait(bar_stage_full + st, (j / C::STAGES) & 1, ctl, 0x712)) break;
+          if (j > 0 && !mbar_wait(bar_s_free, (j - 1) & 1, ctl, 0x713)) break;
+          tc_fence_after();
+          const uint32_t b1 = stage0 + st * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
+          const uint64_t da1 = kmaj | ((a1 >> 4) & 0x3FFFu), da2 = kmaj | ((a2 >> 4) & 0x3FFFu);
+          const uint64_t db1 = kmaj | ((b1 >> 4) & 0x3FFFu), db2 = kmaj | ((b2 >> 4) & 0x3FFFu);
+#pragma unroll
+          for (int kk = 0; kk < DP / 16; ++kk) {
+            const int cb = (kk * 16) / C::CB;
+            const uint32_t in = ((kk * 16) % C::CB) * 2;
+            const uint32_t offa = (cb * C::BLK_M + in) >> 4, offb = (cb * C::BLK_N + in) >> 4;
+            mma_ss(tmem + C::S_COL, da1 + offa, db1 + offb, idesc_s, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::DP_COL, da2 + offa, db2 + offb, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_s_full);
+        }
+        if (j > 0) {
+          if (!mbar_wait(bar_p_full, (j - 1) & 1, ctl, 0x714)) break;
+          tc_fence_after();
+          const int sp = (j - 1) % C::STAGES;
+          const uint32_t b1 = stage0 + sp * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
+          const uint64_t mb1 = mn | ((b1 >> 4) & 0x3FFFu), mb2 = mn | ((b2 >> 4) & 0x3FFFu);
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            const uint32_t off = (kk * 16 * C::ROW_BYTES) >> 4;
+            const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
+            mma_ts(tmem + C::ACC_COL, tmem + C::DS_COL + kk * 8, mb1 + off, idesc_acc, acc);
+            if (KV) mma_ts(tmem + C::ACC_COL + DP, tmem + C::P_COL + kk * 8, mb2 + off, idesc_acc, acc);
+          }
+          mma_commit(bar_pv_done);
+          mma_commit(bar_stage_empty + sp);
+        }
+      }
+      // The epilogue waits on acc_done: every MMA issued has completed (also after an abort).
+      if (rg.n > 0)
+        mma_commit(bar_acc_done);
+      else
+        mbar_arrive(bar_acc_done);
+      bwd_drain(bar_acc_done, 0, w.wait_limit_ns);
+    }
+  } else {
+    // ==================================================================== element-wise (warps 0-7)
+    const int grp = warp >> 2;           // 0: columns 0-31, 1: columns 32-63
+    const int row = (warp & 3) * 32 + lane;
+    const int tid = threadIdx.x;         // 0..255
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int fixed_pos = rg.m0 + row;
+    const long long win = w.causal ? w.window : 0;
+    // Per-row statistics of the fixed rows (dQ instance): LSE log2(e) and D = dO . O.
+    float row_l2 = INFINITY, row_d = 0.f;
+    if (!KV && fixed_pos < w.n_q) {
+      const float L = w.lse[(static_cast<long long>(rg.b) * w.H + rg.hf) * w.n_q + fixed_pos];
+      row_l2 = (L == -INFINITY) ? INFINITY : L * 1.4426950408889634f;
+      const uint4* po = reinterpret_cast<const uint4*>(w.o + rg.b * w.o_sb + rg.hf * w.o_sh + fixed_pos * w.o_st);
+      const uint4* pd = reinterpret_cast<const uint4*>(w.d_o + rg.b * w.do_sb + rg.hf * w.do_sh + fixed_pos * w.do_st);
+      float acc = 0.f;
+      for (int c = 0; c < w.d / 8; ++c) {
+        const uint4 a = po[c], bb = pd[c];
+        const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
+          acc = fmaf(fx.x, fy.x, acc);
+          acc = fmaf(fx.y, fy.y, acc);
+        }
+      }
+      row_d = acc;
+    }
+    bool ok = true;
+    int g = 0, t = rg.tb;
+    for (int j = 0; ok && j < rg.n; ++j) {
+      const int st = j % C::STAGES;
+      const int t0 = t * C::BN;            // first streamed row of the tile
+      const int hs = KV ? rg.hf * w.qpk + g : rg.hf / w.qpk;
+      if (KV) {
+        // D and LSE log2(e) of the tile's 64 query rows: 4 threads per row, each a quarter of
+        // the row's 16-byte chunks of the staged O and dO tiles.  Both tiles share one swizzled
+        // layout, so pairing the same physical chunks pairs the same elements.
+        if (!(ok = bwd_wait(bar_stage_full + st, (j / C::STAGES) & 1, ctl, 0x721))) break;
+        const int c = tid >> 2, part = tid & 3;
+        constexpr int NCH = DP / 32;            // chunks per thread
+        constexpr int CPR = C::CB / 8;          // chunks per row of one column block
+        const uint8_t* sdo = sStage + st * C::STAGE_BYTES + C::TILE_BYTES;
+        const uint8_t* so = sdo + C::TILE_BYTES;
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          const int k = part * NCH + i;
+          const int off = (k / CPR) * C::BLK_N + c * C::ROW_BYTES + (k % CPR) * 16;
+          const uint4 a = *reinterpret_cast<const uint4*>(so + off);
+          const uint4 bb = *reinterpret_cast<const uint4*>(sdo + off);
+          const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+          const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
+            acc = fmaf(fx.x, fy.x, acc);
+            acc = fmaf(fx.y, fy.y, acc);
+          }
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (part == 0) {
+          const int qi = t0 + c;
+          float l2 = INFINITY;  // rows past the end (and empty rows) get P = 0
+          if (qi < w.n_q) {
+            const float L = w.lse[(static_cast<long long>(rg.b) * w.H + hs) * w.n_q + qi];
+            if (L != -INFINITY) l2 = L * 1.4426950408889634f;
+          }
+          s_lse2[(j & 1) * C::BN + c] = l2;
+          s_dd[(j & 1) * C::BN + c] = acc;
+        }
+        mbar_arrive(bar_stage_empty + st);  // done with this stage's O tile
+        mbar_arrive(bar_stats + (j & 1));
+      }
+      // S and dP of this tile's 32 columns of the thread's row.
+      if (!(ok = bwd_wait(bar_s_full, j & 1, ctl, 0x722))) break;
+      tc_fence_after();
+      uint32_t sv[32], pv[32];
+      tmem_ld32(lane_addr + C::S_COL + 32 * grp, sv);
+      tmem_ld32(lane_addr + C::DP_COL + 32 * grp, pv);
+      tmem_ld_wait(sv);
+      reg_pin32(pv);
+      tc_fence_before();
+      mbar_arrive(bar_s_free);
+      // Visible columns i (0..31 of this half) satisfy lo <= i < hi.
+      const int base = t0 + 32 * grp;
+      int lo = 0, hi = 32;
+      bool masked;
+      if (KV) {
+        // fixed row = key at fixed_pos; column = query at base + i.
+        masked = w.causal && (t0 < rg.m0 + C::BM - 1 || (win > 0 && t0 + C::BN - 1 - rg.m0 >= win));
+        if (masked) {
+          lo = fixed_pos - base;                                        // query >= key
+          if (win > 0) hi = static_cast<int>(min(32LL, fixed_pos - base + win));  // query < key + win
+        }
+      } else {
+        // fixed row = query at fixed_pos; column = key at base + i.
+        masked = (t0 + C::BN > w.n_kv) ||
+                 (w.causal && (t0 + C::BN - 1 > rg.m0 || (win > 0 && rg.m0 + C::BM - 1 - t0 >= win)));
+        if (masked) {
+          hi = min(32, w.n_kv - base);
+          if (w.causal) {
+            hi = min(hi, fixed_pos - base + 1);                          // key <= query
+            if (win > 0) lo = static_cast<int>(max(0LL, fixed_pos - win + 1 - base));  // key > query - win
+          }
+        }
+      }
+      if (KV && !(ok = bwd_wait(bar_stats + (j & 1), (j >> 1) & 1, ctl, 0x723))) break;
+      const float* l2v = s_lse2 + (j & 1) * C::BN + 32 * grp;
+      const float* ddv = s_dd + (j & 1) * C::BN + 32 * grp;
+      uint32_t pp[16], dd[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        float p[2], ds[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float l2 = KV ? l2v[i + u] : row_l2;
+          const float dcol = KV ? ddv[i + u] : row_d;
+          float e = bwd_ex2(fmaf(__uint_as_float(sv[i + u]), w.scale_log2, -l2));
+          if (masked && (i + u < lo || i + u >= hi)) e = 0.f;
+          p[u] = e;
+          ds[u] = e * (__uint_as_float(pv[i + u]) - dcol);
+        }
+        pp[i / 2] = bf16x2_bits(p[0], p[1]);
+        dd[i / 2] = bf16x2_bits(ds[0], ds[1]);
+      }
+      if (j > 0 && !(ok = bwd_wait(bar_pv_done, (j - 1) & 1, ctl, 0x724))) break;
+      tc_fence_after();
+      if (KV) tmem_st16(lane_addr + C::P_COL + 16 * grp, pp);
+      tmem_st16(lane_addr + C::DS_COL + 16 * grp, dd);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p_full);
+      if (++t == rg.te) {
+        t = rg.tb;
+        ++g;
+      }
+    }
+    // ================================================================== epilogue
+    const bool have = ok && rg.n > 0 && bwd_wait(bar_acc_done, 0, ctl, 0x725);
+    if (rg.n == 0 || have) {
+      tc_fence_after();
+      const int n_rows = KV ? w.n_kv : w.n_q;
+      const bool row_ok = fixed_pos < n_rows;
+      constexpr int CH = DP / 32;  // 32-column chunks per accumulator
+#pragma unroll 1
+      for (int q = grp; q < C::NACC * CH; q += 2) {
+        const int a = q / CH, ch = q % CH;
+        uint32_t v[32];
+        if (rg.n > 0) {
+          tmem_ld32(lane_addr + C::ACC_COL + a * DP + ch * 32, v);
+          tmem_ld_wait(v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (!row_ok) continue;
+        const float f = (a == 0) ? w.scale : 1.f;
+        float* dst = (a == 0) ? w.out1 + rg.b * w.o1_sb + rg.hf * w.o1_sh + fixed_pos * w.o1_st
+                              : w.out2 + rg.b * w.o2_sb + rg.hf * w.o2_sh + fixed_pos * w.o2_st;
+        const int c0 = ch * 32;
+        const int nc = min(32, w.d - c0);
+        if (nc == 32 && (reinterpret_cast<uintptr_t>(dst + c0) & 15) == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + c0 + i) =
+                make_float4(f * __uint_as_float(v[i]), f * __uint_as_float(v[i + 1]),
+                            f * __uint_as_float(v[i + 2]), f * __uint_as_float(v[i + 3]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nc) dst[c0 + i] = f * __uint_as_float(v[i]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace ra

@@ -7,6 +7,10 @@
 #include "ra_common.cuh"
 
 namespace ra {
+struct BwdTcWork;
+}
+
+namespace ra {
 
 cudaError_t launch_fmha_dp32(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
                              int n_steps, int epi, int sms, cudaStream_t stream);
@@ -14,5 +18,15 @@ cudaError_t launch_fmha_dp64(const CUtensorMap& mq, const CUtensorMap& mk, const
                              int n_steps, int epi, int sms, cudaStream_t stream);
 cudaError_t launch_fmha_dp128(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
                               int n_steps, int epi, int sms, cudaStream_t stream);
+
+// Tensor maps of the tensor-core backward: 128-row boxes for the fixed operands of a CTA,
+// 64-row boxes for the streamed tiles.
+struct BwdMaps {
+  CUtensorMap q128, k128, v128, do128;
+  CUtensorMap q64, k64, v64, do64, o64;
+};
+cudaError_t launch_bwd_dp32(const BwdMaps& m, const BwdTcWork& wq, const BwdTcWork& wkv, cudaStream_t stream);
+cudaError_t launch_bwd_dp64(const BwdMaps& m, const BwdTcWork& wq, const BwdTcWork& wkv, cudaStream_t stream);
+cudaError_t launch_bwd_dp128(const BwdMaps& m, const BwdTcWork& wq, const BwdTcWork& wkv, cudaStream_t stream);
 
 }  // namespace ra
