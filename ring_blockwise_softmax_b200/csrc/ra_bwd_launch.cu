@@ -10,18 +10,30 @@
 
 namespace ra {
 
+template <class C, class K>
+static cudaError_t launch_kernel(K kern, bool kv, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b1,
+                                 const CUtensorMap& b2, const CUtensorMap& b3, const BwdTcWork& w,
+                                 cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int rows = kv ? w.n_kv : w.n_q;
+  const dim3 grid((rows + C::BM - 1) / C::BM, kv ? w.H_kv : w.H, w.B);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(a1, a2, b1, b2, b3, w);
+  return cudaGetLastError();
+}
+
+// The warpgroup ping-pong kernel where each warpgroup's P and dS have their own tensor-memory
+// columns; the column-split kernel where they would have to overwrite S and dP (the dK/dV
+// instance at DP = 128), which measured faster there.
 template <bool KV>
 static cudaError_t launch_bwd_one(const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b1,
                                   const CUtensorMap& b2, const CUtensorMap& b3, const BwdTcWork& w,
                                   cudaStream_t stream) {
-  using C = BwdCfg<RA_BWD_DP, KV>;
-  auto kern = attn_bwd_sm100<RA_BWD_DP, KV>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  const int rows = KV ? w.n_kv : w.n_q;
-  const dim3 grid((rows + C::BM - 1) / C::BM, KV ? w.H_kv : w.H, w.B);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(a1, a2, b1, b2, b3, w);
-  return cudaGetLastError();
+  if constexpr (BwdCfg<RA_BWD_DP, KV>::ALIAS)
+    return launch_kernel<BwdCfgSplit<RA_BWD_DP, KV>>(attn_bwd_sm100_split<RA_BWD_DP, KV>, KV, a1, a2, b1, b2, b3, w,
+                                                     stream);
+  else
+    return launch_kernel<BwdCfg<RA_BWD_DP, KV>>(attn_bwd_sm100<RA_BWD_DP, KV>, KV, a1, a2, b1, b2, b3, w, stream);
 }
 
 #define RA_CAT2(a, b) a##b

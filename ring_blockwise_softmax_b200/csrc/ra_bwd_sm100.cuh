@@ -26,11 +26,12 @@
 // S and dP here are the transposes of each other's roles in the two instances, so both use the
 // forward's operand forms unchanged.  No atomics: every gradient element has one owner.
 //
-// Roles (320 threads): warps 0-7 element-wise (thread = tensor-memory lane (warp % 4) * 32 +
-// lane; warps 0-3 take columns 0-31 of a tile, warps 4-7 columns 32-63) and, at the end, the
-// epilogue; warp 8 TMA producer (and tensor-memory allocation); warp 9 MMA issuer.  The issuer
-// starts S, dP of tile j + 1 as soon as the element-wise warps hold those of tile j in
-// registers, so the tensor core works while they compute.  Every wait is bounded.
+// Roles (320 threads): two element-wise warpgroups (warps 0-3 and 4-7) take alternate streamed
+// tiles, thread = tensor-memory lane (warp % 4) * 32 + lane, all 64 columns of its row; each
+// warpgroup has its own (S, dP) buffer and P, dS columns in tensor memory, so one computes while
+// the other waits on its loads, stores and barriers.  Warp 8 is the TMA producer (and allocates
+// tensor memory), warp 9 the MMA issuer: it starts S, dP of tile j + 2 as soon as warpgroup j % 2
+// holds tile j in registers.  At the end the eight warps run the epilogue.  Every wait is bounded.
 #pragma once
 
 #include "ra_common.cuh"
@@ -75,21 +76,33 @@ struct BwdCfg {
   static constexpr int TILE_BYTES = BN * DP * 2;
   static constexpr int NSTREAM = KV ? 3 : 2;
   static constexpr int STAGE_BYTES = NSTREAM * TILE_BYTES;
-  static constexpr int STAGES_FIT = (192 * 1024 - 2 * FIX_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = (220 * 1024 - 2 * FIX_BYTES) / STAGE_BYTES;  // of 227 KB
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   static_assert(STAGES >= 2, "shared memory holds fewer than two stages");
   static constexpr int NACC = KV ? 2 : 1;
-  // Tensor-memory columns (512 allocated): S, dP (fp32), P, dS (bf16 pairs), ACC1, ACC2.
+  // Tensor-memory columns (512 allocated).  Warpgroup g: (S, dP) buffer at g * 128 (S in its
+  // first 64 columns, dP in the next 64) and P, dS (bf16 pairs, 32 columns each) at
+  // P_COL(g), DS_COL(g); ACC1, ACC2 (DP columns each) from ACC_COL.  The dK/dV instance at
+  // DP = 128 has no room for separate P, dS columns: they overwrite the first 32 columns of the
+  // warpgroup's S and dP once those are in registers (ALIAS), so the next S, dP of that buffer
+  // waits for the products that read them.
+  static constexpr bool ALIAS = NACC * DP > 128;
+  static constexpr int SB_STRIDE = 128;
   static constexpr int S_COL = 0;
   static constexpr int DP_COL = 64;
-  static constexpr int P_COL = 128;
-  static constexpr int DS_COL = 160;
-  static constexpr int ACC_COL = 256;
+  static constexpr int ACC_COL = ALIAS ? 256 : 384;
+  __host__ __device__ static constexpr int P_COL(int g) { return ALIAS ? g * SB_STRIDE : 256 + g * 64; }
+  __host__ __device__ static constexpr int DS_COL(int g) { return ALIAS ? g * SB_STRIDE + 64 : 256 + g * 64 + 32; }
   static_assert(ACC_COL + NACC * DP <= 512, "tensor memory overflow");
-  // Barriers: fixed_full, stage_full[S], stage_empty[S], s_full, s_free, p_full, pv_done,
-  // acc_done, stats_ready[2].
-  static constexpr int NBAR = 1 + 2 * STAGES + 5 + 2;
-  static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + NBAR * 8 + 16 + 4 * BN * 4;
+  // Without ALIAS the issuer starts S(j + 2) before the products of tile j, which needs the stage
+  // of tile j + 2 loaded while tile j's is still held: three stages.
+  static_assert(ALIAS || STAGES >= 3, "the look-ahead needs a third stage");
+  // Barriers: fixed_full, stage_full[S], stage_empty[S], s_full[2], s_free[2], p_full[2],
+  // pv_done[2], acc_done, stats[2][2] (per warpgroup and slot).
+  static constexpr int NBAR = 1 + 2 * STAGES + 8 + 1 + 4;
+  static constexpr int BAR_BYTES = (NBAR * 8 + 15) / 16 * 16;
+  // + tensor-memory slot and abort flag (16 B) + statistics [2 warpgroups][2 slots][BN] float2.
+  static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + BAR_BYTES + 16 + 4 * BN * 8;
   static constexpr int THREADS = 320;
 };
 
@@ -155,6 +168,13 @@ __device__ __forceinline__ void reg_pin32(uint32_t (&r)[32]) {
                  "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 
+// Waits use the suspending try_wait (mbar_wait): spinning on the non-blocking test measured slower
+// here, both for the issuer and for the element-wise warps.
+__device__ __forceinline__ bool bwd_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, const WaitCtl& ctl,
+                                          unsigned site) {
+  return mbar_wait(b0, p0, ctl, site) && (b1 == nullptr || mbar_wait(b1, p1, ctl, site + 1));
+}
+
 __device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, unsigned site) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctl, site));
 }
@@ -180,16 +200,16 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bar_fixed = bars;
   uint64_t* bar_stage_full = bars + 1;
   uint64_t* bar_stage_empty = bar_stage_full + C::STAGES;
-  uint64_t* bar_s_full = bar_stage_empty + C::STAGES;
-  uint64_t* bar_s_free = bar_s_full + 1;
-  uint64_t* bar_p_full = bar_s_free + 1;
-  uint64_t* bar_pv_done = bar_p_full + 1;
-  uint64_t* bar_acc_done = bar_pv_done + 1;
-  uint64_t* bar_stats = bar_acc_done + 1;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_stats + 2);
+  uint64_t* bar_s_full = bar_stage_empty + C::STAGES;  // [2] per warpgroup
+  uint64_t* bar_s_free = bar_s_full + 2;               // [2]
+  uint64_t* bar_p_full = bar_s_free + 2;               // [2]
+  uint64_t* bar_pv_done = bar_p_full + 2;              // [2]
+  uint64_t* bar_acc_done = bar_pv_done + 2;
+  uint64_t* bar_stats = bar_acc_done + 1;  // [2 warpgroups][2 slots]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* s_lse2 = reinterpret_cast<float*>(tmem_slot + 4);  // [2][BN]  LSE log2(e) of streamed rows (KV)
-  float* s_dd = s_lse2 + 2 * C::BN;                          // [2][BN]  D of streamed rows (KV)
+  // [2][2][BN] (LSE log2(e), D) of streamed rows (dK/dV instance); 16-byte aligned.
+  float2* s_st = reinterpret_cast<float2*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -201,15 +221,16 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(bar_fixed, 1);
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(bar_stage_full + i, 1);
-      mbar_init(bar_stage_empty + i, KV ? 1 + 256 : 1);  // MMA commit (+ the D readers of O)
+      mbar_init(bar_stage_empty + i, KV ? 1 + 4 : 1);  // MMA commit (+ the 4 warps reading O)
     }
-    mbar_init(bar_s_full, 1);
-    mbar_init(bar_s_free, 256);
-    mbar_init(bar_p_full, 256);
-    mbar_init(bar_pv_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_s_full + i, 1);
+      mbar_init(bar_s_free + i, 4);  // one arrival per warp of the warpgroup
+      mbar_init(bar_p_full + i, 4);
+      mbar_init(bar_pv_done + i, 1);
+    }
     mbar_init(bar_acc_done, 1);
-    mbar_init(bar_stats + 0, 256);
-    mbar_init(bar_stats + 1, 256);
+    for (int i = 0; i < 4; ++i) mbar_init(bar_stats + i, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -274,41 +295,498 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t mn = make_smem_desc(0, C::BLK_N, C::ATOM_BYTES, C::SWZ);
       const uint32_t a1 = smem_addr(sFix), a2 = a1 + C::FIX_BYTES;
       const uint32_t stage0 = smem_addr(sStage);
-      bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
-      for (int j = 0; ok && j <= rg.n; ++j) {
-        if (j < rg.n) {
-          const int st = j % C::STAGES;
-          if (!mbar_wait(bar_stage_full + st, (j / C::STAGES) & 1, ctl, 0x712)) break;
-          if (j > 0 && !mbar_wait(bar_s_free, (j - 1) & 1, ctl, 0x713)) break;
-          tc_fence_after();
-          const uint32_t b1 = stage0 + st * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
-          const uint64_t da1 = kmaj | ((a1 >> 4) & 0x3FFFu), da2 = kmaj | ((a2 >> 4) & 0x3FFFu);
-          const uint64_t db1 = kmaj | ((b1 >> 4) & 0x3FFFu), db2 = kmaj | ((b2 >> 4) & 0x3FFFu);
+      // S, dP of tile jj into the buffer of warpgroup jj % 2, once the tile's stage has landed and
+      // the warpgroup holds its previous tile (jj - 2) in registers; with ALIAS also once the
+      // products of tile jj - 2 have read that buffer's P, dS.
+      auto issue_s = [&](int jj) -> bool {
+        const int st = jj % C::STAGES, b = jj & 1;
+        const uint32_t ph = ((jj >> 1) - 1) & 1;
+        if (!bwd_wait2(bar_stage_full + st, (jj / C::STAGES) & 1, jj >= 2 ? bar_s_free + b : nullptr, ph, ctl,
+                       0x712))
+          return false;
+        if (C::ALIAS && jj >= 2 && !mbar_wait(bar_pv_done + b, ph, ctl, 0x715)) return false;
+        tc_fence_after();
+        const uint32_t b1 = stage0 + st * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
+        const uint64_t da1 = kmaj | ((a1 >> 4) & 0x3FFFu), da2 = kmaj | ((a2 >> 4) & 0x3FFFu);
+        const uint64_t db1 = kmaj | ((b1 >> 4) & 0x3FFFu), db2 = kmaj | ((b2 >> 4) & 0x3FFFu);
+        const uint32_t col = tmem + b * C::SB_STRIDE;
 #pragma unroll
-          for (int kk = 0; kk < DP / 16; ++kk) {
-            const int cb = (kk * 16) / C::CB;
-            const uint32_t in = ((kk * 16) % C::CB) * 2;
-            const uint32_t offa = (cb * C::BLK_M + in) >> 4, offb = (cb * C::BLK_N + in) >> 4;
-            mma_ss(tmem + C::S_COL, da1 + offa, db1 + offb, idesc_s, kk > 0 ? 1u : 0u);
-            mma_ss(tmem + C::DP_COL, da2 + offa, db2 + offb, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar_s_full);
+        for (int kk = 0; kk < DP / 16; ++kk) {
+          const int cb = (kk * 16) / C::CB;
+          const uint32_t in = ((kk * 16) % C::CB) * 2;
+          const uint32_t offa = (cb * C::BLK_M + in) >> 4, offb = (cb * C::BLK_N + in) >> 4;
+          mma_ss(col + C::S_COL, da1 + offa, db1 + offb, idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(col + C::DP_COL, da2 + offa, db2 + offb, idesc_s, kk > 0 ? 1u : 0u);
         }
-        if (j > 0) {
-          if (!mbar_wait(bar_p_full, (j - 1) & 1, ctl, 0x714)) break;
-          tc_fence_after();
-          const int sp = (j - 1) % C::STAGES;
-          const uint32_t b1 = stage0 + sp * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
-          const uint64_t mb1 = mn | ((b1 >> 4) & 0x3FFFu), mb2 = mn | ((b2 >> 4) & 0x3FFFu);
+        mma_commit(bar_s_full + b);
+        return true;
+      };
+      // ACC1 += dS B1 (and ACC2 += P B2) of tile jj, once its P and dS are in tensor memory; then
+      // its stage and the warpgroup's P, dS columns are released.
+      auto issue_acc = [&](int jj) -> bool {
+        const int b = jj & 1;
+        if (!mbar_wait(bar_p_full + b, (jj >> 1) & 1, ctl, 0x714)) return false;
+        tc_fence_after();
+        const int sp = jj % C::STAGES;
+        const uint32_t b1 = stage0 + sp * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
+        const uint64_t mb1 = mn | ((b1 >> 4) & 0x3FFFu), mb2 = mn | ((b2 >> 4) & 0x3FFFu);
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk) {
-            const uint32_t off = (kk * 16 * C::ROW_BYTES) >> 4;
-            const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
-            mma_ts(tmem + C::ACC_COL, tmem + C::DS_COL + kk * 8, mb1 + off, idesc_acc, acc);
-            if (KV) mma_ts(tmem + C::ACC_COL + DP, tmem + C::P_COL + kk * 8, mb2 + off, idesc_acc, acc);
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          const uint32_t off = (kk * 16 * C::ROW_BYTES) >> 4;
+          const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+          mma_ts(tmem + C::ACC_COL, tmem + C::DS_COL(b) + kk * 8, mb1 + off, idesc_acc, acc);
+          if (KV) mma_ts(tmem + C::ACC_COL + DP, tmem + C::P_COL(b) + kk * 8, mb2 + off, idesc_acc, acc);
+        }
+        mma_commit(bar_pv_done + b);
+        mma_commit(bar_stage_empty + sp);
+        return true;
+      };
+      bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
+      if (ok) ok = issue_s(0);
+      if (ok && rg.n > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < rg.n; ++j) {
+        if (C::ALIAS) {
+          if (!issue_acc(j)) break;
+          if (j + 2 < rg.n && !issue_s(j + 2)) break;
+        } else {
+          // S(j + 2) first: it only needs warpgroup j % 2 to hold S(j), so it runs while that
+          // warpgroup computes tile j.
+          if (j + 2 < rg.n && !issue_s(j + 2)) break;
+          if (!issue_acc(j)) break;
+        }
+      }
+      // The epilogue waits on acc_done: every MMA issued has completed (also after an abort).
+      if (rg.n > 0)
+        mma_commit(bar_acc_done);
+      else
+        mbar_arrive(bar_acc_done);
+      bwd_drain(bar_acc_done, 0, w.wait_limit_ns);
+    }
+  } else {
+    // ==================================================================== element-wise (warps 0-7)
+    const int grp = warp >> 2;  // warpgroup: streamed tiles j with j % 2 == grp
+    const int row = (warp & 3) * 32 + lane;
+    const int tid = threadIdx.x & 127;  // thread within the warpgroup
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t sbuf = lane_addr + grp * C::SB_STRIDE;
+    const int fixed_pos = rg.m0 + row;
+    const long long win = w.causal ? w.window : 0;
+    // Per-row statistics of the fixed rows (dQ instance): LSE log2(e) and D = dO . O.
+    float row_l2 = INFINITY, row_d = 0.f;
+    if (!KV && fixed_pos < w.n_q) {
+      const float L = w.lse[(static_cast<long long>(rg.b) * w.H + rg.hf) * w.n_q + fixed_pos];
+      row_l2 = (L == -INFINITY) ? INFINITY : L * 1.4426950408889634f;
+      const uint4* po = reinterpret_cast<const uint4*>(w.o + rg.b * w.o_sb + rg.hf * w.o_sh + fixed_pos * w.o_st);
+      const uint4* pd = reinterpret_cast<const uint4*>(w.d_o + rg.b * w.do_sb + rg.hf * w.do_sh + fixed_pos * w.do_st);
+      float acc = 0.f;
+      for (int c = 0; c < w.d / 8; ++c) {
+        const uint4 a = po[c], bb = pd[c];
+        const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
+          acc = fmaf(fx.x, fy.x, acc);
+          acc = fmaf(fx.y, fy.y, acc);
+        }
+      }
+      row_d = acc;
+    }
+    // Statistics of streamed query rows (dK/dV instance): D and LSE log2(e) of the 64 rows of the
+    // warpgroup's tile, into its slot k & 1 (k = the warpgroup's tile count).  Two threads per
+    // row, each half of the row's 16-byte chunks of the staged O and dO tiles (both tiles share
+    // one swizzled layout, so the same physical chunks pair the same elements).  A row's LSE is
+    // loaded one tile of the warpgroup ahead.
+    const int sc = tid >> 1, part = tid & 1;
+    auto lse_of = [&](int gg, int tt) -> float {
+      const int qi = tt * C::BN + sc;
+      const int hq = rg.hf * w.qpk + gg;
+      return qi < w.n_q ? w.lse[(static_cast<long long>(rg.b) * w.H + hq) * w.n_q + qi] : -INFINITY;
+    };
+    auto stats = [&](int jj, int kk, float L) -> bool {
+      const int st = jj % C::STAGES;
+      if (!bwd_wait(bar_stage_full + st, (jj / C::STAGES) & 1, ctl, 0x721)) return false;
+      constexpr int NCH = DP / 16;    // chunks per thread
+      constexpr int CPR = C::CB / 8;  // chunks per row of one column block
+      const uint8_t* sdo = sStage + st * C::STAGE_BYTES + C::TILE_BYTES;
+      const uint8_t* so = sdo + C::TILE_BYTES;
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int k = part * NCH + i;
+        const int off = (k / CPR) * C::BLK_N + sc * C::ROW_BYTES + (k % CPR) * 16;
+        const uint4 a = *reinterpret_cast<const uint4*>(so + off);
+        const uint4 bb = *reinterpret_cast<const uint4*>(sdo + off);
+        const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
+          acc = fmaf(fx.x, fy.x, acc);
+          acc = fmaf(fx.y, fy.y, acc);
+        }
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      // Rows past the end (LSE -inf here) and empty rows get LSE log2(e) = +inf, so P = 0.
+      if (part == 0)
+        s_st[(grp * 2 + (kk & 1)) * C::BN + sc] =
+            make_float2(L == -INFINITY ? INFINITY : L * 1.4426950408889634f, acc);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_stage_empty + st);  // this warp is done with the stage's O tile
+        mbar_arrive(bar_stats + grp * 2 + (kk & 1));
+      }
+      return true;
+    };
+    auto advance = [&](int& gg, int& tt) {
+      if (++tt == rg.te) {
+        tt = rg.tb;
+        ++gg;
+      }
+    };
+    bool ok = true;
+    int g = 0, t = rg.tb;  // head and tile of tile j
+    if (grp == 1) advance(g, t);
+    int gn = g, tn = t;    // head and tile of tile j + 2
+    advance(gn, tn);
+    advance(gn, tn);
+    float lse_cur = (KV && part == 0 && grp < rg.n) ? lse_of(g, t) : 0.f;
+    int k = 0;  // tiles of this warpgroup so far
+    for (int j = grp; ok && j < rg.n; j += 2, ++k) {
+      const int t0 = t * C::BN;  // first streamed row of the tile
+      float lse_next = 0.f;
+      if (KV) {
+        if (part == 0 && j + 2 < rg.n) lse_next = lse_of(gn, tn);
+        if (!(ok = stats(j, k, lse_cur))) break;
+      }
+      if (!(ok = bwd_wait(bar_s_full + grp, k & 1, ctl, 0x722))) break;
+      if (KV && !(ok = bwd_wait(bar_stats + grp * 2 + (k & 1), (k >> 1) & 1, ctl, 0x723))) break;
+      tc_fence_after();
+      const float4* stv = reinterpret_cast<const float4*>(s_st + (grp * 2 + (k & 1)) * C::BN);
+      uint32_t pp[32], dd[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sv[32], pv[32];
+        tmem_ld32(sbuf + C::S_COL + 32 * h, sv);
+        tmem_ld32(sbuf + C::DP_COL + 32 * h, pv);
+        tmem_ld_wait(sv);
+        reg_pin32(pv);
+        // Visible columns i (0..31 of this half) satisfy lo <= i < hi.
+        const int base = t0 + 32 * h;
+        int lo = 0, hi = 32;
+        bool masked;
+        if (KV) {
+          // fixed row = key at fixed_pos; column = query at base + i.
+          masked = w.causal && (t0 < rg.m0 + C::BM - 1 || (win > 0 && t0 + C::BN - 1 - rg.m0 >= win));
+          if (masked) {
+            lo = fixed_pos - base;                                                  // query >= key
+            if (win > 0) hi = static_cast<int>(min(32LL, fixed_pos - base + win));  // query < key + win
           }
-          mma_commit(bar_pv_done);
-          mma_commit(bar_stage_empty + sp);
+        } else {
+          // fixed row = query at fixed_pos; column = key at base + i.
+          masked = (t0 + C::BN > w.n_kv) ||
+                   (w.causal && (t0 + C::BN - 1 > rg.m0 || (win > 0 && rg.m0 + C::BM - 1 - t0 >= win)));
+          if (masked) {
+            hi = min(32, w.n_kv - base);
+            if (w.causal) {
+              hi = min(hi, fixed_pos - base + 1);                                        // key <= query
+              if (win > 0) lo = static_cast<int>(max(0LL, fixed_pos - win + 1 - base));  // key > query - win
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float4 cs = make_float4(row_l2, row_d, row_l2, row_d);  // (LSE log2(e), D) of columns i, i + 1
+          if (KV) cs = stv[16 * h + i / 2];
+          float e0 = bwd_ex2(fmaf(__uint_as_float(sv[i]), w.scale_log2, -cs.x));
+          float e1 = bwd_ex2(fmaf(__uint_as_float(sv[i + 1]), w.scale_log2, -cs.z));
+          if (masked) {
+            if (i < lo || i >= hi) e0 = 0.f;
+            if (i + 1 < lo || i + 1 >= hi) e1 = 0.f;
+          }
+          pp[16 * h + i / 2] = bf16x2_bits(e0, e1);
+          dd[16 * h + i / 2] = bf16x2_bits(e0 * (__uint_as_float(pv[i]) - cs.y), e1 * (__uint_as_float(pv[i + 1]) - cs.w));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_s_free + grp);
+      // The warpgroup's P, dS columns are free once the products of its previous tile are done.
+      if (k > 0 && !(ok = bwd_wait(bar_pv_done + grp, (k - 1) & 1, ctl, 0x724))) break;
+      tc_fence_after();
+      if (KV) tmem_st32(lane_addr + C::P_COL(grp), pp);
+      tmem_st32(lane_addr + C::DS_COL(grp), dd);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full + grp);
+      lse_cur = lse_next;
+      advance(g, t);
+      advance(g, t);
+      advance(gn, tn);
+      advance(gn, tn);
+    }
+    // ================================================================== epilogue
+    const bool have = ok && rg.n > 0 && bwd_wait(bar_acc_done, 0, ctl, 0x725);
+    if (rg.n == 0 || have) {
+      tc_fence_after();
+      const int n_rows = KV ? w.n_kv : w.n_q;
+      const bool row_ok = fixed_pos < n_rows;
+      constexpr int CH = DP / 32;  // 32-column chunks per accumulator
+#pragma unroll 1
+      for (int q = grp; q < C::NACC * CH; q += 2) {
+        const int a = q / CH, ch = q % CH;
+        uint32_t v[32];
+        if (rg.n > 0) {
+          tmem_ld32(lane_addr + C::ACC_COL + a * DP + ch * 32, v);
+          tmem_ld_wait(v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (!row_ok) continue;
+        const float f = (a == 0) ? w.scale : 1.f;
+        float* dst = (a == 0) ? w.out1 + rg.b * w.o1_sb + rg.hf * w.o1_sh + fixed_pos * w.o1_st
+                              : w.out2 + rg.b * w.o2_sb + rg.hf * w.o2_sh + fixed_pos * w.o2_st;
+        const int c0 = ch * 32;
+        const int nc = min(32, w.d - c0);
+        if (nc == 32 && (reinterpret_cast<uintptr_t>(dst + c0) & 15) == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + c0 + i) =
+                make_float4(f * __uint_as_float(v[i]), f * __uint_as_float(v[i + 1]),
+                            f * __uint_as_float(v[i + 2]), f * __uint_as_float(v[i + 3]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nc) dst[c0 + i] = f * __uint_as_float(v[i]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Column-split variant, used where the two warpgroups' P and dS do not fit beside their (S, dP)
+// buffers and the accumulators (the dK/dV instance at DP = 128): both warpgroups work on the same
+// tile, warps 0-3 on its columns 0-31 and warps 4-7 on columns 32-63, with one (S, dP) buffer
+// that the issuer refills as soon as every warp holds the current tile in registers.  Same
+// arithmetic, operands and products as attn_bwd_sm100.
+// ---------------------------------------------------------------------------------------------
+template <int DP, bool KV>
+struct BwdCfgSplit {
+  static_assert(DP == 32 || DP == 64 || DP == 128, "padded head dim must be 32, 64 or 128");
+  static constexpr int BM = 128;  // fixed rows (tensor-memory lanes)
+  static constexpr int BN = 64;   // rows of a streamed tile (tensor-memory columns of S, dP)
+  static constexpr int CB = (DP == 32) ? 32 : 64;  // columns per TMA box / swizzle span
+  static constexpr int NCB = DP / CB;
+  static constexpr int ROW_BYTES = CB * 2;
+  static constexpr uint32_t SWZ = (DP == 32) ? kSwizzle64B : kSwizzle128B;
+  static constexpr int ATOM_BYTES = 8 * ROW_BYTES;
+  static constexpr int BLK_M = BM * ROW_BYTES;  // one column block of a fixed operand
+  static constexpr int BLK_N = BN * ROW_BYTES;  // one column block of a streamed operand
+  static constexpr int FIX_BYTES = BM * DP * 2;
+  static constexpr int TILE_BYTES = BN * DP * 2;
+  static constexpr int NSTREAM = KV ? 3 : 2;
+  static constexpr int STAGE_BYTES = NSTREAM * TILE_BYTES;
+  static constexpr int STAGES_FIT = (192 * 1024 - 2 * FIX_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
+  static_assert(STAGES >= 2, "shared memory holds fewer than two stages");
+  static constexpr int NACC = KV ? 2 : 1;
+  // Tensor-memory columns (512 allocated): NSB buffers of (S, dP) (fp32, 64 columns each), P and
+  // dS (bf16 pairs, 32 columns each), ACC1 and ACC2 (DP columns each).  Two (S, dP) buffers let
+  // the issuer compute the tile after next while the element-wise warps work; the dK/dV instance
+  // at DP = 128 has room for one.
+  static constexpr int NSB = (NACC * DP + 384 <= 512) ? 2 : 1;
+  static constexpr int SB_STRIDE = 128;  // columns between (S, dP) buffers
+  static constexpr int S_COL = 0;
+  static constexpr int DP_COL = 64;
+  static constexpr int P_COL = NSB * SB_STRIDE;
+  static constexpr int DS_COL = P_COL + 32;
+  static constexpr int ACC_COL = NSB == 2 ? 384 : 256;
+  static_assert(ACC_COL + NACC * DP <= 512, "tensor memory overflow");
+  static_assert(NSB == 1 || STAGES >= 3, "a second (S, dP) buffer needs a third stage in flight");
+  // Barriers: fixed_full, stage_full[S], stage_empty[S], s_full[2], s_free[2], p_full, pv_done,
+  // acc_done, stats_ready[2].
+  static constexpr int NBAR = 1 + 2 * STAGES + 7 + 2;
+  static_assert((NBAR * 8) % 16 == 0, "statistics buffer must stay 16-byte aligned");
+  static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + NBAR * 8 + 16 + 4 * BN * 4;
+  static constexpr int THREADS = 320;
+};
+
+template <int DP, bool KV>
+__global__ void __launch_bounds__(320, 1)
+    attn_bwd_sm100_split(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
+                   const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
+                   const __grid_constant__ CUtensorMap tm_b3, const BwdTcWork w) {
+  using C = BwdCfgSplit<DP, KV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sFix = smem;                        // A1 | A2
+  uint8_t* sStage = smem + 2 * C::FIX_BYTES;   // STAGES x (B1 | B2 [| B3])
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + C::STAGES * C::STAGE_BYTES);
+  uint64_t* bar_fixed = bars;
+  uint64_t* bar_stage_full = bars + 1;
+  uint64_t* bar_stage_empty = bar_stage_full + C::STAGES;
+  uint64_t* bar_s_full = bar_stage_empty + C::STAGES;  // [2], one per (S, dP) buffer
+  uint64_t* bar_s_free = bar_s_full + 2;               // [2]
+  uint64_t* bar_p_full = bar_s_free + 2;
+  uint64_t* bar_pv_done = bar_p_full + 1;
+  uint64_t* bar_acc_done = bar_pv_done + 1;
+  uint64_t* bar_stats = bar_acc_done + 1;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_stats + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // [2][BN] (LSE log2(e), D) of streamed rows (dK/dV instance); 16-byte aligned.
+  float2* s_st = reinterpret_cast<float2*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  WaitCtl ctl{abort_flag, w.wait_limit_ns, w.dev_status};
+  const BwdRange rg = bwd_range<KV>(w);
+  const int nt = rg.te - rg.tb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_fixed, 1);
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(bar_stage_full + i, 1);
+      mbar_init(bar_stage_empty + i, KV ? 1 + 8 : 1);  // MMA commit (+ the 8 warps reading O)
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_s_full + i, 1);
+      mbar_init(bar_s_free + i, 8);  // one arrival per element-wise warp
+    }
+    mbar_init(bar_p_full, 8);
+    mbar_init(bar_pv_done, 1);
+    mbar_init(bar_acc_done, 1);
+    mbar_init(bar_stats + 0, 8);
+    mbar_init(bar_stats + 1, 8);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    if (lane == 0) {
+      tma_prefetch_map(&tm_a1);
+      tma_prefetch_map(&tm_a2);
+      tma_prefetch_map(&tm_b1);
+      tma_prefetch_map(&tm_b2);
+      if (KV) tma_prefetch_map(&tm_b3);
+    }
+    __syncwarp();
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0 && rg.n > 0) {
+      // ================================================================ TMA producer
+      mbar_arrive_expect_tx(bar_fixed, 2 * C::FIX_BYTES);
+#pragma unroll
+      for (int cb = 0; cb < C::NCB; ++cb) {
+        tma_load_5d(sFix + cb * C::BLK_M, &tm_a1, bar_fixed, cb * C::CB, rg.m0, 0, rg.hf, rg.b);
+        tma_load_5d(sFix + C::FIX_BYTES + cb * C::BLK_M, &tm_a2, bar_fixed, cb * C::CB, rg.m0, 0, rg.hf, rg.b);
+      }
+      int g = 0, t = rg.tb, j = 0;
+      for (; j < rg.n; ++j) {
+        const int st = j % C::STAGES;
+        if (j >= C::STAGES && !mbar_wait(bar_stage_empty + st, ((j / C::STAGES) - 1) & 1, ctl, 0x701)) break;
+        const int hs = KV ? rg.hf * w.qpk + g : rg.hf / w.qpk;  // streamed head
+        uint8_t* dst = sStage + st * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(bar_stage_full + st, C::STAGE_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < C::NCB; ++cb) {
+          tma_load_5d(dst + cb * C::BLK_N, &tm_b1, bar_stage_full + st, cb * C::CB, t * C::BN, 0, hs, rg.b);
+          tma_load_5d(dst + C::TILE_BYTES + cb * C::BLK_N, &tm_b2, bar_stage_full + st, cb * C::CB, t * C::BN, 0,
+                      hs, rg.b);
+          if (KV)
+            tma_load_5d(dst + 2 * C::TILE_BYTES + cb * C::BLK_N, &tm_b3, bar_stage_full + st, cb * C::CB,
+                        t * C::BN, 0, hs, rg.b);
+        }
+        if (++t == rg.te) {
+          t = rg.tb;
+          ++g;
+        }
+      }
+      // No TMA write may still be in flight when the CTA exits.
+      bwd_drain(bar_fixed, 0, w.wait_limit_ns);
+      for (int i = (j > C::STAGES ? j - C::STAGES : 0); i < j; ++i)
+        bwd_drain(bar_stage_full + i % C::STAGES, (i / C::STAGES) & 1, w.wait_limit_ns);
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      // ================================================================ MMA issuer
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, C::BN, 0, 0);
+      constexpr uint32_t idesc_acc = make_idesc_bf16(128, DP, 0, 1);
+      const uint64_t kmaj = make_smem_desc(0, 16, C::ATOM_BYTES, C::SWZ);
+      const uint64_t mn = make_smem_desc(0, C::BLK_N, C::ATOM_BYTES, C::SWZ);
+      const uint32_t a1 = smem_addr(sFix), a2 = a1 + C::FIX_BYTES;
+      const uint32_t stage0 = smem_addr(sStage);
+      // S, dP of tile jj into buffer jj % NSB, once its stage has landed and the element-wise
+      // warps hold the buffer's previous tile in registers.
+      auto issue_s = [&](int jj) -> bool {
+        const int st = jj % C::STAGES, b = jj % C::NSB;
+        if (!bwd_wait2(bar_stage_full + st, (jj / C::STAGES) & 1, jj >= C::NSB ? bar_s_free + b : nullptr,
+                       ((jj / C::NSB) - 1) & 1, ctl, 0x712))
+          return false;
+        tc_fence_after();
+        const uint32_t b1 = stage0 + st * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
+        const uint64_t da1 = kmaj | ((a1 >> 4) & 0x3FFFu), da2 = kmaj | ((a2 >> 4) & 0x3FFFu);
+        const uint64_t db1 = kmaj | ((b1 >> 4) & 0x3FFFu), db2 = kmaj | ((b2 >> 4) & 0x3FFFu);
+        const uint32_t col = tmem + b * C::SB_STRIDE;
+#pragma unroll
+        for (int kk = 0; kk < DP / 16; ++kk) {
+          const int cb = (kk * 16) / C::CB;
+          const uint32_t in = ((kk * 16) % C::CB) * 2;
+          const uint32_t offa = (cb * C::BLK_M + in) >> 4, offb = (cb * C::BLK_N + in) >> 4;
+          mma_ss(col + C::S_COL, da1 + offa, db1 + offb, idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(col + C::DP_COL, da2 + offa, db2 + offb, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s_full + b);
+        return true;
+      };
+      // ACC1 += dS B1 (and ACC2 += P B2) of tile jj, once its P and dS are in tensor memory; then
+      // its stage and the P, dS columns are released.
+      auto issue_acc = [&](int jj) -> bool {
+        if (!mbar_wait(bar_p_full, jj & 1, ctl, 0x714)) return false;
+        tc_fence_after();
+        const int sp = jj % C::STAGES;
+        const uint32_t b1 = stage0 + sp * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
+        const uint64_t mb1 = mn | ((b1 >> 4) & 0x3FFFu), mb2 = mn | ((b2 >> 4) & 0x3FFFu);
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          const uint32_t off = (kk * 16 * C::ROW_BYTES) >> 4;
+          const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+          mma_ts(tmem + C::ACC_COL, tmem + C::DS_COL + kk * 8, mb1 + off, idesc_acc, acc);
+          if (KV) mma_ts(tmem + C::ACC_COL + DP, tmem + C::P_COL + kk * 8, mb2 + off, idesc_acc, acc);
+        }
+        mma_commit(bar_pv_done);
+        mma_commit(bar_stage_empty + sp);
+        return true;
+      };
+      bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
+      if (C::NSB == 1) {
+        // S(j + 1) as soon as S(j) is in registers, then the products of tile j.
+        for (int j = 0; ok && j <= rg.n; ++j) {
+          if (j < rg.n && !issue_s(j)) break;
+          if (j > 0 && !issue_acc(j - 1)) break;
+        }
+      } else {
+        // Two tiles ahead: S(j + 2) right after the products of tile j.
+        if (ok) ok = issue_s(0);
+        if (ok && rg.n > 1) ok = issue_s(1);
+        for (int j = 0; ok && j < rg.n; ++j) {
+          if (!issue_acc(j)) break;
+          if (j + 2 < rg.n && !issue_s(j + 2)) break;
         }
       }
       // The epilogue waits on acc_done: every MMA issued has completed (also after an abort).
@@ -347,63 +825,80 @@ __global__ void __launch_bounds__(320, 1)
       }
       row_d = acc;
     }
-    bool ok = true;
-    int g = 0, t = rg.tb;
-    for (int j = 0; ok && j < rg.n; ++j) {
-      const int st = j % C::STAGES;
-      const int t0 = t * C::BN;            // first streamed row of the tile
-      const int hs = KV ? rg.hf * w.qpk + g : rg.hf / w.qpk;
-      if (KV) {
-        // D and LSE log2(e) of the tile's 64 query rows: 4 threads per row, each a quarter of
-        // the row's 16-byte chunks of the staged O and dO tiles.  Both tiles share one swizzled
-        // layout, so pairing the same physical chunks pairs the same elements.
-        if (!(ok = bwd_wait(bar_stage_full + st, (j / C::STAGES) & 1, ctl, 0x721))) break;
-        const int c = tid >> 2, part = tid & 3;
-        constexpr int NCH = DP / 32;            // chunks per thread
-        constexpr int CPR = C::CB / 8;          // chunks per row of one column block
-        const uint8_t* sdo = sStage + st * C::STAGE_BYTES + C::TILE_BYTES;
-        const uint8_t* so = sdo + C::TILE_BYTES;
-        float acc = 0.f;
+    // Statistics of streamed query rows (dK/dV instance), one tile ahead of their use: D and
+    // LSE log2(e) of tile jj's 64 rows go to buffer jj & 1 as interleaved pairs.  Four threads per
+    // row, each a quarter of the row's 16-byte chunks of the staged O and dO tiles (both tiles
+    // share one swizzled layout, so the same physical chunks pair the same elements); the row's
+    // LSE is loaded one tile before it is needed.
+    const int sc = tid >> 2, part = tid & 3;
+    auto lse_of = [&](int gg, int tt) -> float {
+      const int qi = tt * C::BN + sc;
+      const int hq = rg.hf * w.qpk + gg;
+      return qi < w.n_q ? w.lse[(static_cast<long long>(rg.b) * w.H + hq) * w.n_q + qi] : -INFINITY;
+    };
+    auto stats = [&](int jj, float L) -> bool {
+      const int st = jj % C::STAGES;
+      if (!bwd_wait(bar_stage_full + st, (jj / C::STAGES) & 1, ctl, 0x721)) return false;
+      constexpr int NCH = DP / 32;    // chunks per thread
+      constexpr int CPR = C::CB / 8;  // chunks per row of one column block
+      const uint8_t* sdo = sStage + st * C::STAGE_BYTES + C::TILE_BYTES;
+      const uint8_t* so = sdo + C::TILE_BYTES;
+      float acc = 0.f;
 #pragma unroll
-        for (int i = 0; i < NCH; ++i) {
-          const int k = part * NCH + i;
-          const int off = (k / CPR) * C::BLK_N + c * C::ROW_BYTES + (k % CPR) * 16;
-          const uint4 a = *reinterpret_cast<const uint4*>(so + off);
-          const uint4 bb = *reinterpret_cast<const uint4*>(sdo + off);
-          const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
-          const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&bb);
+      for (int i = 0; i < NCH; ++i) {
+        const int k = part * NCH + i;
+        const int off = (k / CPR) * C::BLK_N + sc * C::ROW_BYTES + (k % CPR) * 16;
+        const uint4 a = *reinterpret_cast<const uint4*>(so + off);
+        const uint4 bb = *reinterpret_cast<const uint4*>(sdo + off);
+        const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&bb);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
-            acc = fmaf(fx.x, fy.x, acc);
-            acc = fmaf(fx.y, fy.y, acc);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
+          acc = fmaf(fx.x, fy.x, acc);
+          acc = fmaf(fx.y, fy.y, acc);
         }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (part == 0) {
-          const int qi = t0 + c;
-          float l2 = INFINITY;  // rows past the end (and empty rows) get P = 0
-          if (qi < w.n_q) {
-            const float L = w.lse[(static_cast<long long>(rg.b) * w.H + hs) * w.n_q + qi];
-            if (L != -INFINITY) l2 = L * 1.4426950408889634f;
-          }
-          s_lse2[(j & 1) * C::BN + c] = l2;
-          s_dd[(j & 1) * C::BN + c] = acc;
-        }
-        mbar_arrive(bar_stage_empty + st);  // done with this stage's O tile
-        mbar_arrive(bar_stats + (j & 1));
       }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      // Rows past the end (LSE -inf here) and empty rows get LSE log2(e) = +inf, so P = 0.
+      if (part == 0) s_st[(jj & 1) * C::BN + sc] = make_float2(L == -INFINITY ? INFINITY : L * 1.4426950408889634f, acc);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_stage_empty + st);  // this warp is done with the stage's O tile
+        mbar_arrive(bar_stats + (jj & 1));
+      }
+      return true;
+    };
+    bool ok = true;
+    int g = 0, t = rg.tb;    // head and tile of tile j
+    int gn = 0, tn = rg.tb;  // head and tile of the next tile whose statistics are due
+    auto advance = [&](int& gg, int& tt) {
+      if (++tt == rg.te) {
+        tt = rg.tb;
+        ++gg;
+      }
+    };
+    if (KV && rg.n > 0) {
+      ok = stats(0, part == 0 ? lse_of(0, rg.tb) : 0.f);
+      advance(gn, tn);
+    }
+    for (int j = 0; ok && j < rg.n; ++j) {
+      const int t0 = t * C::BN;  // first streamed row of the tile
+      float lse_next = 0.f;
+      if (KV && part == 0 && j + 1 < rg.n) lse_next = lse_of(gn, tn);
       // S and dP of this tile's 32 columns of the thread's row.
-      if (!(ok = bwd_wait(bar_s_full, j & 1, ctl, 0x722))) break;
+      const int sb = j % C::NSB;
+      if (!(ok = bwd_wait(bar_s_full + sb, (j / C::NSB) & 1, ctl, 0x722))) break;
       tc_fence_after();
       uint32_t sv[32], pv[32];
-      tmem_ld32(lane_addr + C::S_COL + 32 * grp, sv);
-      tmem_ld32(lane_addr + C::DP_COL + 32 * grp, pv);
+      tmem_ld32(lane_addr + sb * C::SB_STRIDE + C::S_COL + 32 * grp, sv);
+      tmem_ld32(lane_addr + sb * C::SB_STRIDE + C::DP_COL + 32 * grp, pv);
       tmem_ld_wait(sv);
       reg_pin32(pv);
       tc_fence_before();
-      mbar_arrive(bar_s_free);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_s_free + sb);
       // Visible columns i (0..31 of this half) satisfy lo <= i < hi.
       const int base = t0 + 32 * grp;
       int lo = 0, hi = 32;
@@ -412,7 +907,7 @@ __global__ void __launch_bounds__(320, 1)
         // fixed row = key at fixed_pos; column = query at base + i.
         masked = w.causal && (t0 < rg.m0 + C::BM - 1 || (win > 0 && t0 + C::BN - 1 - rg.m0 >= win));
         if (masked) {
-          lo = fixed_pos - base;                                        // query >= key
+          lo = fixed_pos - base;                                                  // query >= key
           if (win > 0) hi = static_cast<int>(min(32LL, fixed_pos - base + win));  // query < key + win
         }
       } else {
@@ -422,29 +917,26 @@ __global__ void __launch_bounds__(320, 1)
         if (masked) {
           hi = min(32, w.n_kv - base);
           if (w.causal) {
-            hi = min(hi, fixed_pos - base + 1);                          // key <= query
+            hi = min(hi, fixed_pos - base + 1);                                        // key <= query
             if (win > 0) lo = static_cast<int>(max(0LL, fixed_pos - win + 1 - base));  // key > query - win
           }
         }
       }
       if (KV && !(ok = bwd_wait(bar_stats + (j & 1), (j >> 1) & 1, ctl, 0x723))) break;
-      const float* l2v = s_lse2 + (j & 1) * C::BN + 32 * grp;
-      const float* ddv = s_dd + (j & 1) * C::BN + 32 * grp;
+      const float4* stv = reinterpret_cast<const float4*>(s_st + (j & 1) * C::BN + 32 * grp);
       uint32_t pp[16], dd[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
-        float p[2], ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const float l2 = KV ? l2v[i + u] : row_l2;
-          const float dcol = KV ? ddv[i + u] : row_d;
-          float e = bwd_ex2(fmaf(__uint_as_float(sv[i + u]), w.scale_log2, -l2));
-          if (masked && (i + u < lo || i + u >= hi)) e = 0.f;
-          p[u] = e;
-          ds[u] = e * (__uint_as_float(pv[i + u]) - dcol);
+        float4 cs = make_float4(row_l2, row_d, row_l2, row_d);  // (LSE log2(e), D) of columns i, i + 1
+        if (KV) cs = stv[i / 2];
+        float e0 = bwd_ex2(fmaf(__uint_as_float(sv[i]), w.scale_log2, -cs.x));
+        float e1 = bwd_ex2(fmaf(__uint_as_float(sv[i + 1]), w.scale_log2, -cs.z));
+        if (masked) {
+          if (i < lo || i >= hi) e0 = 0.f;
+          if (i + 1 < lo || i + 1 >= hi) e1 = 0.f;
         }
-        pp[i / 2] = bf16x2_bits(p[0], p[1]);
-        dd[i / 2] = bf16x2_bits(ds[0], ds[1]);
+        pp[i / 2] = bf16x2_bits(e0, e1);
+        dd[i / 2] = bf16x2_bits(e0 * (__uint_as_float(pv[i]) - cs.y), e1 * (__uint_as_float(pv[i + 1]) - cs.w));
       }
       if (j > 0 && !(ok = bwd_wait(bar_pv_done, (j - 1) & 1, ctl, 0x724))) break;
       tc_fence_after();
@@ -452,10 +944,12 @@ __global__ void __launch_bounds__(320, 1)
       tmem_st16(lane_addr + C::DS_COL + 16 * grp, dd);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar_p_full);
-      if (++t == rg.te) {
-        t = rg.tb;
-        ++g;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full);
+      advance(g, t);
+      if (KV && j + 1 < rg.n) {
+        if (!(ok = stats(j + 1, lse_next))) break;
+        advance(gn, tn);
       }
     }
     // ================================================================== epilogue
