@@ -168,7 +168,13 @@ ra_status_t ra_lse_merge_n(const float* const* o_parts, const float* const* lse_
  * dq fp32 [B,H,Nq,d], dk, dv fp32 [B,H_kv,Nk,d]; all overwritten.  scale <= 0 selects 1/sqrt(d).
  * window: 0, or with causal the forward's sliding window.  The backward of ra_ring_fwd (either
  * layout or schedule) is this call on the same full tensors: the ring computes the same function
- * of global positions.  Arithmetic is fp32 (SIMT kernels), inputs fp32 or bf16. */
+ * of global positions.
+ * bf16 inputs whose q, k, v, o, d_o satisfy the forward's TMA rules (16-byte aligned base,
+ * strides multiples of 8 elements, d % 8 == 0) run on the tensor cores: P and dS are rounded to
+ * bf16 before the products dv = P^T d_o, dk = dS^T q, dq = dS k (fp32 accumulation), so each
+ * gradient element errs by at most ~2^-8 times the same sums taken over absolute values.
+ * fp32 inputs (and bf16 tensors outside those rules) use fp32 SIMT kernels.  Two launches on
+ * `stream`, no workspace.  Errors: RA_ERR_INVALID_ARG for shape / dtype / window mismatches. */
 ra_status_t ra_attn_bwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
                         const ra_tensor_t* o, const float* lse, const ra_tensor_t* d_o,
                         const ra_tensor_t* dq, const ra_tensor_t* dk, const ra_tensor_t* dv,
