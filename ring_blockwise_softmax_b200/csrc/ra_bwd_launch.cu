@@ -22,14 +22,14 @@ static cudaError_t launch_kernel(K kern, bool kv, const CUtensorMap& a1, const C
   return cudaGetLastError();
 }
 
-// The warpgroup ping-pong kernel where each warpgroup's P and dS have their own tensor-memory
-// columns; the column-split kernel where they would have to overwrite S and dP (the dK/dV
-// instance at DP = 128), which measured faster there.
+// The warpgroup ping-pong kernel wherever each warpgroup's (S, dP) buffer and P, dS columns fit
+// beside the accumulators; the column-split kernel for the dK/dV instance at DP = 128, where they
+// do not (writing P, dS over S, dP instead measured slower there).
 template <bool KV>
 static cudaError_t launch_bwd_one(const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b1,
                                   const CUtensorMap& b2, const CUtensorMap& b3, const BwdTcWork& w,
                                   cudaStream_t stream) {
-  if constexpr (BwdCfg<RA_BWD_DP, KV>::ALIAS)
+  if constexpr (KV && RA_BWD_DP == 128)
     return launch_kernel<BwdCfgSplit<RA_BWD_DP, KV>>(attn_bwd_sm100_split<RA_BWD_DP, KV>, KV, a1, a2, b1, b2, b3, w,
                                                      stream);
   else

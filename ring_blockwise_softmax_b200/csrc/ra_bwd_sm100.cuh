@@ -29,7 +29,8 @@
 // Roles (320 threads): two element-wise warpgroups (warps 0-3 and 4-7) take alternate streamed
 // tiles, thread = tensor-memory lane (warp % 4) * 32 + lane, all 64 columns of its row; each
 // warpgroup has its own (S, dP) buffer and P, dS columns in tensor memory, so one computes while
-// the other waits on its loads, stores and barriers.  Warp 8 is the TMA producer (and allocates
+// the other waits on its loads, stores and barriers.  (The dK/dV instance at DP = 128 lacks the
+// tensor memory for that and runs attn_bwd_sm100_split, further below.)  Warp 8 is the TMA producer (and allocates
 // tensor memory), warp 9 the MMA issuer: it starts S, dP of tile j + 2 as soon as warpgroup j % 2
 // holds tile j in registers.  At the end the eight warps run the epilogue.  Every wait is bounded.
 #pragma once
@@ -82,21 +83,19 @@ struct BwdCfg {
   static constexpr int NACC = KV ? 2 : 1;
   // Tensor-memory columns (512 allocated).  Warpgroup g: (S, dP) buffer at g * 128 (S in its
   // first 64 columns, dP in the next 64) and P, dS (bf16 pairs, 32 columns each) at
-  // P_COL(g), DS_COL(g); ACC1, ACC2 (DP columns each) from ACC_COL.  The dK/dV instance at
-  // DP = 128 has no room for separate P, dS columns: they overwrite the first 32 columns of the
-  // warpgroup's S and dP once those are in registers (ALIAS), so the next S, dP of that buffer
-  // waits for the products that read them.
-  static constexpr bool ALIAS = NACC * DP > 128;
+  // P_COL(g), DS_COL(g); ACC1, ACC2 (DP columns each) from ACC_COL.  This leaves room for
+  // NACC * DP <= 128: every instance but dK/dV at DP = 128, which runs the column-split kernel
+  // (BwdCfgSplit) instead.
   static constexpr int SB_STRIDE = 128;
   static constexpr int S_COL = 0;
   static constexpr int DP_COL = 64;
-  static constexpr int ACC_COL = ALIAS ? 256 : 384;
-  __host__ __device__ static constexpr int P_COL(int g) { return ALIAS ? g * SB_STRIDE : 256 + g * 64; }
-  __host__ __device__ static constexpr int DS_COL(int g) { return ALIAS ? g * SB_STRIDE + 64 : 256 + g * 64 + 32; }
-  static_assert(ACC_COL + NACC * DP <= 512, "tensor memory overflow");
-  // Without ALIAS the issuer starts S(j + 2) before the products of tile j, which needs the stage
-  // of tile j + 2 loaded while tile j's is still held: three stages.
-  static_assert(ALIAS || STAGES >= 3, "the look-ahead needs a third stage");
+  static constexpr int ACC_COL = 384;
+  __host__ __device__ static constexpr int P_COL(int g) { return 256 + g * 64; }
+  __host__ __device__ static constexpr int DS_COL(int g) { return 256 + g * 64 + 32; }
+  static_assert(ACC_COL + NACC * DP <= 512, "tensor memory overflow: use the column-split kernel");
+  // The issuer starts S(j + 2) before the products of tile j, which needs the stage of tile j + 2
+  // loaded while tile j's is still held: three stages.
+  static_assert(STAGES >= 3, "the look-ahead needs a third stage");
   // Barriers: fixed_full, stage_full[S], stage_empty[S], s_full[2], s_free[2], p_full[2],
   // pv_done[2], acc_done, stats[2][2] (per warpgroup and slot).
   static constexpr int NBAR = 1 + 2 * STAGES + 8 + 1 + 4;
@@ -296,15 +295,12 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t a1 = smem_addr(sFix), a2 = a1 + C::FIX_BYTES;
       const uint32_t stage0 = smem_addr(sStage);
       // S, dP of tile jj into the buffer of warpgroup jj % 2, once the tile's stage has landed and
-      // the warpgroup holds its previous tile (jj - 2) in registers; with ALIAS also once the
-      // products of tile jj - 2 have read that buffer's P, dS.
+      // the warpgroup holds its previous tile (jj - 2) in registers.
       auto issue_s = [&](int jj) -> bool {
         const int st = jj % C::STAGES, b = jj & 1;
-        const uint32_t ph = ((jj >> 1) - 1) & 1;
-        if (!bwd_wait2(bar_stage_full + st, (jj / C::STAGES) & 1, jj >= 2 ? bar_s_free + b : nullptr, ph, ctl,
-                       0x712))
+        if (!bwd_wait2(bar_stage_full + st, (jj / C::STAGES) & 1, jj >= 2 ? bar_s_free + b : nullptr,
+                       ((jj >> 1) - 1) & 1, ctl, 0x712))
           return false;
-        if (C::ALIAS && jj >= 2 && !mbar_wait(bar_pv_done + b, ph, ctl, 0x715)) return false;
         tc_fence_after();
         const uint32_t b1 = stage0 + st * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
         const uint64_t da1 = kmaj | ((a1 >> 4) & 0x3FFFu), da2 = kmaj | ((a2 >> 4) & 0x3FFFu);
@@ -345,15 +341,10 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) ok = issue_s(0);
       if (ok && rg.n > 1) ok = issue_s(1);
       for (int j = 0; ok && j < rg.n; ++j) {
-        if (C::ALIAS) {
-          if (!issue_acc(j)) break;
-          if (j + 2 < rg.n && !issue_s(j + 2)) break;
-        } else {
-          // S(j + 2) first: it only needs warpgroup j % 2 to hold S(j), so it runs while that
-          // warpgroup computes tile j.
-          if (j + 2 < rg.n && !issue_s(j + 2)) break;
-          if (!issue_acc(j)) break;
-        }
+        // S(j + 2) first: it only needs warpgroup j % 2 to hold S(j), so it runs while that
+        // warpgroup computes tile j.
+        if (j + 2 < rg.n && !issue_s(j + 2)) break;
+        if (!issue_acc(j)) break;
       }
       // The epilogue waits on acc_done: every MMA issued has completed (also after an abort).
       if (rg.n > 0)
@@ -471,6 +462,12 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld32(sbuf + C::DP_COL + 32 * h, pv);
         tmem_ld_wait(sv);
         reg_pin32(pv);
+        if (h == 1) {
+          // The whole tile is in registers: the issuer may refill this warpgroup's buffer.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_s_free + grp);
+        }
         // Visible columns i (0..31 of this half) satisfy lo <= i < hi.
         const int base = t0 + 32 * h;
         int lo = 0, hi = 32;
@@ -508,9 +505,6 @@ __global__ void __launch_bounds__(320, 1)
           dd[16 * h + i / 2] = bf16x2_bits(e0 * (__uint_as_float(pv[i]) - cs.y), e1 * (__uint_as_float(pv[i + 1]) - cs.w));
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_s_free + grp);
       // The warpgroup's P, dS columns are free once the products of its previous tile are done.
       if (k > 0 && !(ok = bwd_wait(bar_pv_done + grp, (k - 1) & 1, ctl, 0x724))) break;
       tc_fence_after();
