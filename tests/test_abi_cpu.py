@@ -112,3 +112,34 @@ def test_ring_workspace_size(ra):
     assert ra.ring_workspace_size(q, 8, "stepwise") == rows * 64 * 4 + rows * 4
     with pytest.raises(ra.RaError):
         ra.ring_workspace_size(q, 3, "stepwise")  # 8192 % 3 != 0
+
+
+def test_backward_host_validation(ra):
+    """ra_attn_bwd rejects bad arguments before any CUDA call."""
+    import torch
+
+    lib = ra.lib_handle()
+    q = torch.zeros(1, 4, 32, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 2, 32, 64, dtype=torch.bfloat16)
+    g32 = torch.zeros(1, 4, 32, 64, dtype=torch.float32)
+    gk = torch.zeros(1, 2, 32, 64, dtype=torch.float32)
+    lse = torch.zeros(1, 4, 32, dtype=torch.float32)
+    tq, tk, tg, tgk = (ra.tensor_desc(x) for x in (q, k, g32, gk))
+    lse_p = ctypes.c_void_p(lse.data_ptr())
+
+    def call(dq=tg, dk=tgk, dv=tgk, lse_ptr=lse_p, causal=1, window=0, o=tq, d_o=tq, kk=tk):
+        return lib.ra_attn_bwd(ctypes.byref(tq), ctypes.byref(kk), ctypes.byref(kk), ctypes.byref(o), lse_ptr,
+                               ctypes.byref(d_o), ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv),
+                               ctypes.c_float(0.0), causal, ctypes.c_int64(window), None)
+
+    assert call(lse_ptr=None) == ra.RA_ERR_INVALID_ARG and b"lse is NULL" in lib.ra_last_error()
+    tbad = ra.tensor_desc(torch.zeros(1, 4, 32, 64, dtype=torch.bfloat16))
+    assert call(dq=tbad) == ra.RA_ERR_INVALID_ARG and b"fp32" in lib.ra_last_error()
+    assert call(dq=tgk) == ra.RA_ERR_INVALID_ARG and b"shape of q" in lib.ra_last_error()
+    assert call(dk=tg) == ra.RA_ERR_INVALID_ARG and b"shape of k" in lib.ra_last_error()
+    assert call(causal=0, window=16) == ra.RA_ERR_INVALID_ARG and b"window" in lib.ra_last_error()
+    assert call(window=-1) == ra.RA_ERR_INVALID_ARG
+    to32 = ra.tensor_desc(torch.zeros(1, 4, 32, 64, dtype=torch.float32))
+    assert call(o=to32) == ra.RA_ERR_INVALID_ARG and b"q's dtype" in lib.ra_last_error()
+    k3 = ra.tensor_desc(torch.zeros(1, 3, 32, 64, dtype=torch.bfloat16))
+    assert call(kk=k3) == ra.RA_ERR_INVALID_ARG
