@@ -388,15 +388,18 @@ def test_against_torch_softmax_fp64():
 
 def check_backward(bwd):
     """The backward pass against an independent differentiation of the forward definition:
-    torch autograd in float64 through softmax(scale Q K^T + mask) V (non-causal, causal, and a
-    sliding window), and central finite differences of L = sum(dO * O) on a tiny case."""
+    torch autograd in float64 through softmax(scale Q K^T + mask) V (non-causal, causal, a
+    sliding window, and non-causal with fewer queries than keys), and central finite differences
+    of L = sum(dO * O) on a tiny case."""
     try:
         import torch
     except ImportError:  # pragma: no cover
         return True
-    for n, d, kind in ((40, 16, "full"), (37, 8, "causal"), (30, 12, "window")):
-        rng = np.random.default_rng(n * d)
-        q, k, v, do = (rng.normal(size=(n, d)) for _ in range(4))
+    for n, n_k, d, kind in ((40, 40, 16, "full"), (37, 37, 8, "causal"), (30, 30, 12, "window"),
+                            (23, 41, 8, "full")):
+        rng = np.random.default_rng(n * d + n_k)
+        q, do = (rng.normal(size=(n, d)) for _ in range(2))
+        k, v = (rng.normal(size=(n_k, d)) for _ in range(2))
         scale = 0.7 / math.sqrt(d)
         pos = np.arange(n)
         allowed = None if kind == "full" else A.allowed_mask(pos, pos, True, 5 if kind == "window" else None)
