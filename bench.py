@@ -268,7 +268,8 @@ class OracleSampler:
         self.flops += 4.0 * w.d * float(keys)
 
 
-def cpu_baseline(w, budget_s: float = 12.0, rows_per_step: int = 64):
+def cpu_baseline(w, budget_s: float = 12.0, rows_per_step: int = 64, single_s: float = 3.0):
+    """The oracle on the host's cores (BLAS threads), then the same on one thread for single_s."""
     s = OracleSampler(w, rows_per_step)
     t0 = time.perf_counter()
     n = 0
@@ -276,9 +277,23 @@ def cpu_baseline(w, budget_s: float = 12.0, rows_per_step: int = 64):
         s.step()
         n += 1
     dt = time.perf_counter() - t0
-    return {"value": s.flops / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{n * rows_per_step} query rows ({rows_per_step} seeded uniform rows per chunk, cycling the "
-                      f"{w.B * w.H} heads) of the workload, fp64 numpy oracle, {dt:.1f} s"}
+    out = {"value": s.flops / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{n * rows_per_step} query rows ({rows_per_step} seeded uniform rows per chunk, cycling the "
+                     f"{w.B * w.H} heads) of the workload, fp64 numpy oracle, {dt:.1f} s"}
+    if single_s > 0:
+        from threadpoolctl import threadpool_limits
+
+        with threadpool_limits(limits=1):
+            s.flops = 0.0
+            n1 = 0
+            t1 = time.perf_counter()
+            while time.perf_counter() - t1 < single_s:
+                s.step()
+                n1 += 1
+            dt1 = time.perf_counter() - t1
+        out["single_thread"] = {"value": s.flops / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                                "sample": f"{n1 * rows_per_step} query rows, same sampling, {dt1:.1f} s"}
+    return out
 
 
 def run_reference(args, w):
