@@ -233,11 +233,9 @@ class OracleSampler:
         self.np = np
         self.w = w
         self.rows = rows_per_step
-        # Host copies of the inputs; the oracle widens the exact bf16/fp32 values to fp64.
-        q, k, v = I.make_qkv(w)
-        self.q = q.float().numpy()
-        self.k = k.float().numpy()
-        self.v = v.float().numpy()
+        # Host copies of the inputs (the workload's dtype); the oracle widens the exact bf16/fp32
+        # values of one head at a time to fp64.
+        self.q, self.k, self.v = I.make_qkv(w)
         self.cursor = 0
         self.flops = 0.0
         self.rng = np.random.default_rng(w.seed)
@@ -255,10 +253,10 @@ class OracleSampler:
         rows = np.sort(self.rng.choice(w.N, size=min(self.rows, w.N), replace=False))
         pos = np.arange(w.N)
         hk = oracle.kv_head(h, w.H, self.k.shape[1])  # K/V head (grouped-query K/V)
-        k = self.k[b, hk].astype(np.float64)
-        v = self.v[b, hk].astype(np.float64)
-        oracle.attention_rows(self.q[b, h][rows].astype(np.float64), k, v, w.scale, rows, pos, w.causal,
-                              window=w.window)
+        k = self.k[b, hk].float().numpy().astype(np.float64)
+        v = self.v[b, hk].float().numpy().astype(np.float64)
+        q = self.q[b, h].float().numpy()[rows].astype(np.float64)
+        oracle.attention_rows(q, k, v, w.scale, rows, pos, w.causal, window=w.window)
         if w.window is not None:
             keys = np.minimum(rows + 1, w.window).sum()
         elif w.causal:
@@ -338,6 +336,67 @@ def config_dict(w, args):
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
 
 
+def time_forward(w, args, dev, stream, flush, world, steps: int, warmup: int):
+    """Time `steps` ring-forward steps of workload w (inputs resident in HBM, L2 flushed between
+    steps outside the events).  Returns (mean ms over ranks' max, per-step ms, clocks, launches per
+    step, device tensors)."""
+    import torch
+
+    from ring_blockwise_softmax_b200 import inputs as I
+    from ring_blockwise_softmax_b200 import ra_attn as ra
+
+    q_h, k_h, v_h = I.make_qkv(w)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    assert q.stride() == q_h.stride()
+    B, H, N, d = q.shape
+    o = torch.empty((B, H, N, d), dtype=q.dtype, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ws_bytes = ra.ring_workspace_size(q, w.P, args.schedule)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+
+    def step():
+        ra.ring_fwd(q, k, v, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws, w.window or 0)
+
+    launches = 1 if (args.schedule == "fused" or w.P == 1) else w.P
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ra.get_device_status(stream) == ra.RA_OK
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = max_over_ranks(sum(per_step) / len(per_step), world, dev)
+    status = ra.get_device_status(stream)
+    bufs = {"host": (q_h, k_h, v_h), "dev": (q, k, v), "o": o, "lse": lse, "ws": ws, "step": step}
+    return ms, per_step, clocks.summary(), launches, status, bufs
+
+
+def forward_roofline(w, ms: float, world: int, peak: float, peak_kind: str, launches: int, traffic):
+    value = world * w.flops() / (ms * 1e-3) / 1e12
+    return value, {
+        "bound": "tensor", "kernel": "fmha_fwd_sm100", "achieved": value / world, "peak": peak,
+        "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s", "frac": (value / world) / peak,
+        "traffic": traffic,
+        "note": ("algorithmic FLOPs (4*d per visible query-key pair: 4*B*H*N^2*d, halved when causal; "
+                 "sum_i min(i+1, w) pairs per head with a sliding window w) / summed duration of the "
+                 f"step's {launches} serialised launches (CUDA events on the launch stream)")}
+
+
+def traffic_key(w, backward: bool = False) -> str:
+    key = f"cfg{w.cfg}" + ("" if w.H_kv is None else f"-kv{w.H_kv}") + ("" if w.window is None else f"-w{w.window}")
+    return key + ("-bwd" if backward else "")
+
+
 def run_gpu(args, w):
     import torch
 
@@ -349,59 +408,51 @@ def run_gpu(args, w):
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
     peaks, peak_kind = load_peaks()
-
-    q_h, k_h, v_h = I.make_qkv(w)
-    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
-    assert q.stride() == q_h.stride()
-    B, H, N, d = q.shape
-    o = torch.empty((B, H, N, d), dtype=q.dtype, device=dev)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    ws_bytes = ra.ring_workspace_size(q, w.P, args.schedule)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    peak = peaks["bf16_tflops"]
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        ra.ring_fwd(q, k, v, w.P, w.layout, w.causal, o, lse, 0.0, args.schedule, [stream], ws, w.window or 0)
-
-    launches_per_step = 1 if (args.schedule == "fused" or w.P == 1) else w.P
+    ms, per_step_ms, clk, launches_per_step, status, bufs = time_forward(
+        w, args, dev, stream, flush, world, args.steps, args.warmup)
+    q_h, k_h, v_h = bufs["host"]
+    q, k, v = bufs["dev"]
+    o, lse, ws = bufs["o"], bufs["lse"], bufs["ws"]
+    flops = w.flops()
     if args.backward:
         # Backward of the ring forward = backward on the full tensors (same function of global
         # positions): ra_attn_bwd from the forward's saved O and LSE, dO drawn like the inputs.
-        step()
+        bufs["step"]()
         do_ = I.draw(tuple(q.shape), w.seed, 3, "normal", 1.0, w.dtype).to(dev)
         dq_ = torch.empty(q.shape, dtype=torch.float32, device=dev)
         dk_ = torch.empty(k.shape, dtype=torch.float32, device=dev)
         dv_ = torch.empty(v.shape, dtype=torch.float32, device=dev)
         o_saved, lse_saved = o.clone(), lse.clone()
 
-        def step():  # noqa: F811 - the timed step of the backward mode
+        def bstep():
             ra.attn_bwd(q, k, v, o_saved, lse_saved, do_, dq_, dk_, dv_, 0.0, w.causal, w.window or 0, stream)
 
-        launches_per_step = 2
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert ra.get_device_status(stream) == ra.RA_OK
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        for i in range(args.steps):
-            flush.zero_()
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
+        for _ in range(args.warmup):
+            bstep()
         torch.cuda.synchronize()
-    barrier(world)
-    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms_local = sum(per_step_ms) / len(per_step_ms)
-    ms = max_over_ranks(ms_local, world, dev)
-    status = ra.get_device_status(stream)
-    flops = w.flops() * (2.5 if args.backward else 1.0)  # backward: 5 products of 2*d per pair
+        assert ra.get_device_status(stream) == ra.RA_OK
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clocks_b:
+            for i in range(args.steps):
+                flush.zero_()
+                starts[i].record(stream)
+                bstep()
+                ends[i].record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        ms = max_over_ranks(sum(per_step_ms) / len(per_step_ms), world, dev)
+        status = ra.get_device_status(stream)
+        clk = clocks_b.summary()
+        launches_per_step = 2
+        flops = w.flops() * 2.5  # backward: 5 products of 2*d per pair
     value = world * flops / (ms * 1e-3) / 1e12
 
     # End to end through the public API: pinned host inputs -> device, ring forward, result -> host.
@@ -450,6 +501,10 @@ def run_gpu(args, w):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    del qp, kp, vp, qd, kd, vd, o_host, lse_host, bufs, q, k, v, o, lse, ws
+    if args.backward:
+        del extra_in, grads_host, dq_, dk_, dv_, do_, o_saved, lse_saved
+    torch.cuda.empty_cache()
 
     # Standalone LSE merge of 16 fp32 partials O[1,8,16384,128] + LSE (the k-way merge kernel).
     merge = None
@@ -473,19 +528,49 @@ def run_gpu(args, w):
             b.record(stream)
             times.append((a, b))
         torch.cuda.synchronize()
-        mms = statistics.mean(a.elapsed_time(b) for a, b in times)
+        mms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in times), world, dev)
         mbytes = (kparts + 1) * rows * (dm + 1) * 4
         gbs = mbytes / (mms * 1e-3) / 1e9
         merge = {"kernel": "lse_merge_n_kernel", "workload": "16 x fp32 O[1,8,16384,128] + LSE[1,8,16384]",
                  "algorithmic_bytes": mbytes, "ms": mms, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
-                 "frac": gbs / peaks["hbm_gbs"], "frac_of_8000": gbs / 8000.0}
+                 "frac": gbs / peaks["hbm_gbs"], "frac_of_8000": gbs / 8000.0, "launches": 20}
+        del mo_l, ml_l, out_o, out_l, mo, ml
+        torch.cuda.empty_cache()
+
+    # The other bf16 workloads, each timed the same way (the headline keys stay on the main one).
+    others = {}
+    if not args.backward and args.configs:
+        for c in [int(x) for x in args.configs.split(",") if x.strip()]:
+            if c == w.cfg:
+                continue
+            wc = I.WORKLOADS[c]
+            steps_c = max(3, min(args.steps, args.config_steps))
+            ms_c, per_c, clk_c, l_c, st_c, bufs_c = time_forward(wc, args, dev, stream, flush, world, steps_c,
+                                                                 args.warmup)
+            del bufs_c
+            torch.cuda.empty_cache()
+            v_c, roof_c = forward_roofline(wc, ms_c, world, peak, peak_kind, l_c,
+                                           recorded_traffic(traffic_key(wc), args.schedule))
+            others[f"cfg{c}"] = {
+                "workload": wc.name, "steps": steps_c, "ms_per_step": ms_c, "value": v_c, "unit": "TFLOP/s",
+                "flops_per_step": wc.flops(), "pct_of_spec_bf16_peak": 100.0 * (v_c / world) / SPEC_BF16_TFLOPS,
+                "roofline": roof_c, "mufu_roofline": mufu_roofline(wc, ms_c, world, clk_c),
+                "gpu_launches": l_c * steps_c, "clocks": clk_c, "device_status": ra.status_string(st_c),
+                "step_ms_min": min(per_c), "step_ms_median": statistics.median(per_c)}
 
     if rank != 0:
         return 0
-    peak = peaks["bf16_tflops"]
-    traffic_key = f"cfg{w.cfg}" + ("" if w.H_kv is None else f"-kv{w.H_kv}") + ("" if w.window is None else f"-w{w.window}")
     if args.backward:
-        traffic_key += "-bwd"
+        roof = {"bound": "tensor", "kernel": "attn_bwd_sm100 (dQ + dK/dV instances)", "achieved": value / world,
+                "peak": peak, "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s",
+                "frac": (value / world) / peak,
+                "traffic": args.traffic if args.traffic is not None else recorded_traffic(traffic_key(w, True),
+                                                                                           args.schedule),
+                "note": BWD_NOTE}
+    else:
+        _, roof = forward_roofline(w, ms, world, peak, peak_kind, launches_per_step,
+                                   args.traffic if args.traffic is not None
+                                   else recorded_traffic(traffic_key(w), args.schedule))
     line = {
         "metric": METRIC_BWD if args.backward else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps,
@@ -494,28 +579,20 @@ def run_gpu(args, w):
         "config": config_dict(w, args),
         "pct_of_spec_bf16_peak": 100.0 * (value / world) / SPEC_BF16_TFLOPS,
         "pct_of_measured_bf16_peak": 100.0 * (value / world) / peak,
-        "roofline": {"bound": "tensor",
-                     "kernel": ("attn_bwd_sm100 (dQ + dK/dV instances)" if args.backward else "fmha_fwd_sm100"),
-                     "achieved": value / world, "peak": peak,
-                     "peak_kind": f"{peak_kind} bf16 burst", "unit": "TFLOP/s", "frac": (value / world) / peak,
-                     "traffic": args.traffic if args.traffic is not None else recorded_traffic(traffic_key,
-                                                                                                  args.schedule),
-                     "note": (BWD_NOTE if args.backward else
-                              "algorithmic FLOPs (4*d per visible query-key pair: 4*B*H*N^2*d, halved when causal; "
-                              "sum_i min(i+1, w) pairs per head with a sliding window w) / summed duration of the "
-                              f"step's {launches_per_step} serialised launches (CUDA events on the launch stream)")},
-        "mufu_roofline": None if args.backward else mufu_roofline(w, ms, world, clocks.summary()),
-        "fp32_roofline": (fp32_roofline(value / world, clocks.summary())
-                          if args.backward and w.dtype == "f32" else None),
+        "roofline": roof,
+        "mufu_roofline": None if args.backward else mufu_roofline(w, ms, world, clk),
+        "fp32_roofline": (fp32_roofline(value / world, clk) if args.backward and w.dtype == "f32" else None),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clk,
         "device_status": ra.status_string(status),
         "step_ms_min": min(per_step_ms), "step_ms_median": statistics.median(per_step_ms),
     }
     if merge is not None:
         line["merge"] = merge
+    if others:
+        line["configs"] = others
     if not args.skip_cpu and world == 1 and not args.backward:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
     print(json.dumps(line), flush=True)
@@ -527,7 +604,12 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--config", type=int, default=3,
+                    help="headline workload (default 3: the largest bf16 causal ring, B=1 H=32 N=32768 d=128)")
+    ap.add_argument("--configs", default="2,4,5",
+                    help="other workloads timed in the same run, reported under 'configs' ('' for none)")
+    ap.add_argument("--config-steps", type=int, default=20,
+                    help="timed steps per workload under 'configs' (at most --steps)")
     ap.add_argument("--schedule", choices=["stepwise", "fused"], default="fused")
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--e2e-steps", type=int, default=20)

@@ -29,8 +29,11 @@
  *  - Asynchrony: every compute call only enqueues work on the given stream(s) and returns.  The
  *    return value reports argument and launch errors.  Faults detected on the device (a bounded
  *    wait that ran out) are latched in a device status word read by ra_get_device_status().
- *  - Errors never abort the process.  On a non-RA_OK return nothing has been enqueued, and
- *    ra_last_error() returns a message for the calling thread.
+ *  - Errors never abort the process, and ra_last_error() returns a message for the calling thread.
+ *    On a non-RA_OK return no kernel has been enqueued: every argument, shape and index limit is
+ *    checked before the first launch.  The one exception is RA_ERR_CUDA from the CUDA runtime
+ *    refusing a kernel launch in the middle of a multi-launch ring call (ra_ring_fwd and its
+ *    variants): the launches before it stay queued, and streams[0] is still ordered after them.
  *  - Device pointers must belong to the current CUDA device.
  *
  * Supported inputs
@@ -155,8 +158,6 @@ ra_status_t ra_lse_merge_n(const float* const* o_parts, const float* const* lse_
                            float* o_out, float* lse_out, int64_t rows, int d,
                            ra_stream_t stream);
 
-/* Workspace bytes ra_ring_fwd needs for (q, P, schedule): 0 for RA_RING_FUSED; for
- * RA_RING_STEPWISE an fp32 accumulator of B*H*N*(d+1)*4 bytes (plus alignment). */
 /* Backward pass (extension beyond the forward path the pages' ring method needs): gradients of
  * L = sum(d_o * O) with respect to q, k, v for O = ra_attn_fwd(q, k, v, ..., scale, causal) (or
  * ra_attn_fwd_window with window > 0), with the attention weights recomputed from the forward's
@@ -180,6 +181,8 @@ ra_status_t ra_attn_bwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
                         const ra_tensor_t* dq, const ra_tensor_t* dk, const ra_tensor_t* dv,
                         float scale, int causal, int64_t window, ra_stream_t stream);
 
+/* Workspace bytes ra_ring_fwd needs for (q, P, schedule): 0 for RA_RING_FUSED; for
+ * RA_RING_STEPWISE an fp32 accumulator of B*H*N*(d+1)*4 bytes (plus alignment). */
 ra_status_t ra_ring_workspace_size(const ra_tensor_t* q, int P, int schedule, size_t* bytes);
 
 /* Ring attention over P virtual sequence shards on one GPU (vibe-research page, "Ring
@@ -211,20 +214,23 @@ ra_status_t ra_ring_fwd_window(const ra_tensor_t* q, const ra_tensor_t* k, const
                                int n_streams, void* workspace, size_t workspace_bytes);
 
 /* ra_ring_fwd with the RA_RING_STEPWISE schedule for callers that cannot allocate device memory
- * at the point of the call: code recording a CUDA graph (cudaMalloc cannot be captured), code
- * whose device memory is entirely held by another allocator, or latency-critical paths that
- * must not pay for an allocation's implicit synchronisation.  There is no counterpart on the
- * source pages: this is an interface convenience of this library.
+ * at the point of the call: code inside a host application whose caching allocator already holds
+ * all device memory and offers no scratch interface, services that fix their memory budget at
+ * start-up and allow no allocation afterwards, and latency-critical paths that must not pay for
+ * the implicit device-wide synchronisation of cudaMalloc / cudaFree.  There is no counterpart on
+ * the source pages: this is an interface convenience of this library.
  * The fp32 (O, LSE) accumulator lives in a fixed array of RA_NOALLOC_SCRATCH_BYTES inside the
  * library (held on every device that loads the library, until the process exits); nothing is
  * allocated.  Problems whose accumulator (ra_ring_workspace_size with RA_RING_STEPWISE) exceeds
  * that size are rejected with RA_ERR_WORKSPACE and a message naming both sizes.
- * The first call on each device looks up the array's device address with that device current;
- * make that first call before any stream capture.  All calls on a device share the one array:
- * calls whose work overlaps on the GPU (different streams, or interleaved with ra_ring_fwd_noalloc
- * calls on other threads) race on it, so order them on one stream.  The array keeps the last
- * call's contents; no clearing is needed because ring step 0 overwrites every element the later
- * steps read.  Other arguments and errors as for ra_ring_fwd (one stream). */
+ * Set-up: the first call on each device (and again the first call after the device's context has
+ * been torn down and recreated, e.g. by cudaDeviceReset) looks up the array's device address with
+ * that device current; make that first call before any stream capture.  All calls on a device
+ * share the one array: calls whose work overlaps on the GPU (different streams, or interleaved
+ * with ra_ring_fwd_noalloc calls on other threads) race on it, so order them on one stream.  The
+ * array keeps the last call's contents; no clearing is needed because ring step 0 overwrites
+ * every element the later steps read.  Other arguments and errors as for ra_ring_fwd (one
+ * stream). */
 #define RA_NOALLOC_SCRATCH_BYTES (32u << 20)
 ra_status_t ra_ring_fwd_noalloc(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P,
                                 int layout, int causal, float scale, const ra_tensor_t* o, float* lse,

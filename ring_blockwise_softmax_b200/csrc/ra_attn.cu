@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "ra_attn.h"
 #include "ra_attn_simt.cuh"
@@ -79,10 +80,17 @@ ra_status_t cuda_fail(cudaError_t e, const char* what) {
 // ------------------------------------------------------------------------------------------
 struct DevInfo {
   int major = -1, minor = -1, sms = 0;
-  unsigned int* status = nullptr;  // device address of ra::g_dev_status on this device
+  unsigned int* status = nullptr;  // device address of ra::g_dev_status in the context below
+  unsigned long long ctx = 0;      // context the address was looked up in
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+std::once_flag g_ctx_once;
 
 ra_status_t current_device(DevInfo* out) {
   int dev = 0;
@@ -97,14 +105,17 @@ ra_status_t current_device(DevInfo* out) {
     g_dev[dev].major = p.major;
     g_dev[dev].minor = p.minor;
     g_dev[dev].sms = p.multiProcessorCount;
-    if (p.major == 10 && p.minor == 0) {
+  }
+  if (g_dev[dev].major == 10 && g_dev[dev].minor == 0) {
+    // The status word's address, looked up again whenever the current context is not the one it
+    // was found in (or the context cannot be identified).
+    const unsigned long long ctx = ra::current_context_id();
+    if (g_dev[dev].status == nullptr || ctx == 0 || ctx != g_dev[dev].ctx) {
       void* addr = nullptr;
       e = cudaGetSymbolAddress(&addr, ra::g_dev_status);
-      if (e != cudaSuccess) {
-        g_dev[dev].major = -1;
-        return cuda_fail(e, "cudaGetSymbolAddress(status word)");
-      }
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
       g_dev[dev].status = static_cast<unsigned int*>(addr);
+      g_dev[dev].ctx = ra::current_context_id();
     }
   }
   *out = g_dev[dev];
@@ -250,8 +261,9 @@ int heads_per_group(const ra::AttnWork& w, int elem_bytes) {
   return 1;
 }
 
-ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::AttnWork& w_in, int n_steps, int epi,
-                             int sms, cudaStream_t stream) {
+// Completes a launch's work description (head groups, fast dividers) and checks every limit of
+// the kernels' index arithmetic, without launching anything.
+ra_status_t prepare_attention(const ra_tensor_t* q, const ra::AttnWork& w_in, int n_steps, ra::AttnWork* out) {
   if (w_in.B > 65535 || w_in.H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
   ra::AttnWork w = w_in;
   if (w.H_kv == 0) w.H_kv = w.H;
@@ -276,6 +288,15 @@ ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::A
     if (w.H_kv < 1 || w.H % w.H_kv != 0) return fail(RA_ERR_INVALID_ARG, "H_kv must divide H");
     w.fd_qpk = ra::make_fastdiv(static_cast<unsigned>(w.H / w.H_kv));
   }
+  if (q->dtype != RA_BF16 && static_cast<long long>(w.n_q_tiles) * w.n_r > 2147483647LL)
+    return fail(RA_ERR_UNSUPPORTED, "grid too large");
+  *out = w;
+  return RA_OK;
+}
+
+// Launches a work description completed by prepare_attention.
+ra_status_t launch_prepared(const ra_tensor_t* q, const Maps* maps, const ra::AttnWork& w, int n_steps, int epi,
+                            int sms, cudaStream_t stream) {
   cudaError_t e;
   if (q->dtype == RA_BF16) {
     const int dp = padded_dim(w.d);
@@ -287,7 +308,6 @@ ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::A
       e = ra::launch_fmha_dp128(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream);
   } else {
     const long long gx = static_cast<long long>(w.n_q_tiles) * w.n_r;
-    if (gx > 2147483647LL) return fail(RA_ERR_UNSUPPORTED, "grid too large");
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(w.H), static_cast<unsigned>(w.B));
     const int dp = padded_dim(w.d);
     if (dp == 32)
@@ -300,6 +320,14 @@ ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::A
   }
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return RA_OK;
+}
+
+ra_status_t launch_attention(const ra_tensor_t* q, const Maps* maps, const ra::AttnWork& w_in, int n_steps, int epi,
+                             int sms, cudaStream_t stream) {
+  ra::AttnWork w;
+  ra_status_t st = prepare_attention(q, w_in, n_steps, &w);
+  if (st != RA_OK) return st;
+  return launch_prepared(q, maps, w, n_steps, epi, sms, stream);
 }
 
 void set_operand_ptrs(ra::AttnWork& w, const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v,
@@ -409,6 +437,26 @@ static void launch_merge_n(int G, dim3 grid, cudaStream_t st, const ra::MergePar
 }  // namespace
 
 namespace ra {
+unsigned long long current_context_id() {
+  std::call_once(g_ctx_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 // Lets the library's other translation units report through ra_last_error().
 ra_status_t set_last_error(ra_status_t status, const char* message) { return fail(status, "%s", message); }
 }  // namespace ra
@@ -679,54 +727,80 @@ static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, con
     if ((st = encode_view(&maps.v, shard_view(v, n_local, P, shard_rows, tok_rows), dp)) != RA_OK) return st;
   }
 
-  // Fork the extra streams off streams[0] so the call is ordered after work already queued there.
-  cudaStream_t s0 = reinterpret_cast<cudaStream_t>(streams[0]);
-  cudaEvent_t ev_fork = nullptr;
-  cudaError_t e;
-  if (n_streams > 1) {
-    if ((e = cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "event");
-    if ((e = cudaEventRecord(ev_fork, s0)) != cudaSuccess) {
-      cudaEventDestroy(ev_fork);
-      return cuda_fail(e, "event record");
-    }
-    for (int i = 1; i < n_streams; ++i) {
-      if ((e = cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(streams[i]), ev_fork, 0)) != cudaSuccess) {
-        cudaEventDestroy(ev_fork);
-        return cuda_fail(e, "stream wait");
-      }
-    }
-    cudaEventDestroy(ev_fork);
-  }
-
-  st = RA_OK;
-  for (int i = 0; i < n_streams && st == RA_OK; ++i) {
+  // Every launch of the call is described and checked before the first one is enqueued.
+  struct Launch {
+    ra::AttnWork w;
+    int stream, n_steps, epi;
+  };
+  std::vector<Launch> launches;
+  for (int i = 0; i < n_streams; ++i) {
     ra::AttnWork wi = w;
     wi.r_first = i;
     wi.r_step = n_streams;
     wi.n_r = (P - i + n_streams - 1) / n_streams;
-    cudaStream_t si = reinterpret_cast<cudaStream_t>(streams[i]);
     if (schedule == RA_RING_FUSED || P == 1) {
       wi.ring_step = 0;
-      st = launch_attention(q, &maps, wi, P, ra::kEpiOut, dev.sms, si);
+      launches.push_back({wi, i, P, ra::kEpiOut});
     } else {
-      for (int t = 0; t < P && st == RA_OK; ++t) {
+      for (int t = 0; t < P; ++t) {
         wi.ring_step = t;
-        const int epi = t == 0 ? ra::kEpiPart : (t == P - 1 ? ra::kEpiAccOut : ra::kEpiAcc);
-        st = launch_attention(q, &maps, wi, 1, epi, dev.sms, si);
+        launches.push_back({wi, i, 1, t == 0 ? ra::kEpiPart : (t == P - 1 ? ra::kEpiAccOut : ra::kEpiAcc)});
       }
     }
   }
+  for (Launch& l : launches)
+    if ((st = prepare_attention(q, l.w, l.n_steps, &l.w)) != RA_OK) return st;
 
-  // Join: later work on streams[0] waits for every stream of this call.
-  for (int i = 1; i < n_streams; ++i) {
+  // Events that fork the extra streams off streams[0] (so the call is ordered after work already
+  // queued there) and join them back, created before anything is enqueued.
+  cudaStream_t s0 = reinterpret_cast<cudaStream_t>(streams[0]);
+  std::vector<cudaEvent_t> events;
+  auto destroy_events = [&events] {
+    for (cudaEvent_t ev : events) cudaEventDestroy(ev);
+  };
+  cudaError_t e;
+  for (int i = 0; i < (n_streams > 1 ? n_streams : 0); ++i) {
     cudaEvent_t ev = nullptr;
-    if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "event");
-    e = cudaEventRecord(ev, reinterpret_cast<cudaStream_t>(streams[i]));
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s0, ev, 0);
-    cudaEventDestroy(ev);
-    if (e != cudaSuccess) return cuda_fail(e, "stream join");
+    if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) {
+      destroy_events();
+      return cuda_fail(e, "event");
+    }
+    events.push_back(ev);  // events[0]: fork; events[i >= 1]: join of streams[i]
   }
-  return st == RA_OK ? ok() : st;
+  if (n_streams > 1) {
+    e = cudaEventRecord(events[0], s0);
+    for (int i = 1; i < n_streams && e == cudaSuccess; ++i)
+      e = cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(streams[i]), events[0], 0);
+    if (e != cudaSuccess) {
+      destroy_events();
+      return cuda_fail(e, "stream fork");
+    }
+  }
+
+  // A launch can still fail here only through the CUDA runtime; the streams that already hold
+  // work of this call are joined to streams[0] all the same, and the error is returned.
+  st = RA_OK;
+  std::string launch_error;
+  for (const Launch& l : launches) {
+    st = launch_prepared(q, &maps, l.w, l.n_steps, l.epi, dev.sms, reinterpret_cast<cudaStream_t>(streams[l.stream]));
+    if (st != RA_OK) {
+      launch_error = t_last_error;
+      break;
+    }
+  }
+  for (int i = 1; i < n_streams; ++i) {
+    e = cudaEventRecord(events[i], reinterpret_cast<cudaStream_t>(streams[i]));
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s0, events[i], 0);
+    if (e != cudaSuccess) {
+      destroy_events();
+      return cuda_fail(e, "stream join (kernels of this call may be queued)");
+    }
+  }
+  destroy_events();
+  if (st != RA_OK)
+    return fail(st, "%s (earlier launches of this ring call stay queued, ordered before later work on streams[0])",
+                launch_error.c_str());
+  return ok();
 }
 
 ra_status_t ra_attn_fwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, const ra_tensor_t* o,

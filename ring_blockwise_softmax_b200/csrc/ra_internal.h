@@ -12,6 +12,12 @@ struct BwdTcWork;
 
 namespace ra {
 
+// Identifier of the calling thread's current CUDA context (cuCtxGetId), or 0 when there is none
+// yet or the driver cannot say.  Device addresses of the library's __device__ variables are cached
+// per context: a context torn down and created again (cudaDeviceReset) reloads the module, and
+// the variables may then sit at other addresses.
+unsigned long long current_context_id();
+
 cudaError_t launch_fmha_dp32(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
                              int n_steps, int epi, int sms, cudaStream_t stream);
 cudaError_t launch_fmha_dp64(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,

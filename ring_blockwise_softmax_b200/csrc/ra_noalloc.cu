@@ -2,11 +2,12 @@
 // in a fixed, library-owned device array instead of caller-provided workspace.
 //
 // Who needs it: callers that cannot allocate device memory at the point of the call.  Examples:
-// code running while a CUDA stream is being captured into a graph (cudaMalloc is not a
-// capturable operation), code inside an application whose caching allocator already owns all
-// device memory and exposes no scratch API, and latency-critical paths that must not pay for
-// cudaMalloc's implicit device-wide synchronisation.  The caller still passes the inputs and
-// outputs; only the intermediate (O, LSE) accumulator moves into the library.
+// code running inside a host application whose caching allocator already owns all device memory
+// and exposes no scratch interface (a cudaMalloc there fails, or fragments the pool), services that
+// fix their memory budget at start-up and forbid allocations afterwards, and latency-critical
+// paths that must not pay for the implicit device-wide synchronisation of cudaMalloc / cudaFree.
+// The caller still passes the inputs and outputs; only the intermediate (O, LSE) accumulator
+// moves into the library.
 //
 // The array lives for as long as the library is loaded, on every device that loads it.
 #include <cuda_runtime.h>
@@ -15,6 +16,7 @@
 #include <string>
 
 #include "ra_attn.h"
+#include "ra_internal.h"
 
 namespace ra {
 ra_status_t set_last_error(ra_status_t status, const char* message);  // defined in ra_attn.cu
@@ -25,8 +27,13 @@ namespace {
 // Scratch for the stepwise ring's fp32 (O, LSE) accumulator; its size is RA_NOALLOC_SCRATCH_BYTES.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RA_NOALLOC_SCRATCH_BYTES];
 
+// Device address of g_noalloc_scratch per device ordinal, with the context it was looked up in.
+struct ScratchAddr {
+  void* ptr = nullptr;
+  unsigned long long ctx = 0;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {nullptr};  // device address of g_noalloc_scratch, per device ordinal
+ScratchAddr g_noalloc_addr[64];
 
 ra_status_t noalloc_fail(ra_status_t st, const std::string& msg) { return ra::set_last_error(st, msg.c_str()); }
 
@@ -49,16 +56,21 @@ extern "C" ra_status_t ra_ring_fwd_noalloc(const ra_tensor_t* q, const ra_tensor
   if (dev < 0 || dev >= 64) return noalloc_fail(RA_ERR_UNSUPPORTED, "device ordinal out of range");
   void* ptr = nullptr;
   {
-    // Once per device, with that device current: the symbol's device address (the name itself is
-    // only a host-side stand-in and must never be handed to a kernel).
+    // Set-up, once per device and context, with that device current: the symbol's device address
+    // (the name itself is only a host-side stand-in and must never be handed to a kernel).  The
+    // address is looked up again when the current context is not the one it was found in, e.g.
+    // after cudaDeviceReset, which reloads the module.
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    const unsigned long long ctx = ra::current_context_id();
+    ScratchAddr& a = g_noalloc_addr[dev];
+    if (a.ptr == nullptr || ctx == 0 || ctx != a.ctx) {
       e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
       if (e != cudaSuccess)
         return noalloc_fail(RA_ERR_CUDA, std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(e));
-      g_noalloc_ptr[dev] = ptr;
+      a.ptr = ptr;
+      a.ctx = ra::current_context_id();
     }
-    ptr = g_noalloc_ptr[dev];
+    ptr = a.ptr;
   }
   // Step 0 of the stepwise ring writes every accumulator element that later steps read, so the
   // scratch needs no clearing between calls.

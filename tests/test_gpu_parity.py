@@ -247,12 +247,24 @@ def test_workload4_merge_of_16_partials(ra):
     sel = oracle.sample_rows(rows, 4096, seed=4, must_include=[1, rows - 2])
     ref_o, ref_l = oracle.merge_many(o[:, sel].double().numpy(), lse[:, sel].double().numpy())
     compare(to64(out_o)[sel], to64(out_l)[sel], ref_o, ref_l, "f32", "16-way merge")
-    # pairwise fold with the 2-way kernel gives the same result
+    # Pairwise fold with the 2-way kernel: k - 1 dependent fp32 merges.  Each merge rounds
+    # L = hi + log1p(e^(lo - hi)) once at magnitude |L| (half an ulp, |L| 2^-24) and its log1p /
+    # exp terms (below 1) to within 2^-23; errors already in the inputs pass through with weights
+    # that sum to 1.  So |dLSE| <= (k - 1) 2^-24 (max|L| + 2), and O, whose weights e^(l_i - L) carry
+    # that error in the exponent plus one rounding per merge, |dO| <= (|dLSE| bound +
+    # (k - 1) 2^-23) max|O|.  For this workload: 1.5e-5 and 1.7e-5 (an fp32 emulation of the fold
+    # on the CPU reaches 2.9e-6 and 3.0e-6).  The one-pass k-way kernel above meets the fp32 bounds.
     acc_o, acc_l = o_list[0].clone(), l_list[0].clone()
     for i in range(1, k):
         ra.lse_merge(acc_o, acc_l, o_list[i], l_list[i], acc_o, acc_l)
     torch.cuda.synchronize()
-    compare(to64(acc_o)[sel], to64(acc_l)[sel], ref_o, ref_l, "bf16", "pairwise fold")
+    got_o, got_l = to64(acc_o)[sel], to64(acc_l)[sel]
+    fin = np.isfinite(ref_l)
+    assert np.array_equal(np.isneginf(got_l), ~fin)
+    lse_bound = (k - 1) * 2.0 ** -24 * (np.abs(ref_l[fin]).max() + 2.0)
+    o_bound = (lse_bound + (k - 1) * 2.0 ** -23) * np.abs(ref_o).max()
+    assert np.abs(got_l[fin] - ref_l[fin]).max() <= lse_bound
+    assert np.abs(got_o - ref_o).max() <= o_bound
 
 
 # ------------------------------------------------------------------------------- failure path

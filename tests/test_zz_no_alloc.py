@@ -1,6 +1,7 @@
 """ra_ring_fwd_noalloc: the stepwise ring for callers that cannot allocate device memory (for
-example while capturing a CUDA graph, or when another allocator owns all device memory).  Its
-accumulator lives in a fixed array inside the library instead of caller workspace.
+example when another allocator already owns all device memory, or when a service allows no
+allocation after start-up).  Its accumulator lives in a fixed array inside the library instead of
+caller workspace.
 
 Checked against ra_ring_fwd (same schedule, caller-allocated workspace) within the parity
 tolerances, on two calls in a row (the second call sees the first call's leftover scratch).
