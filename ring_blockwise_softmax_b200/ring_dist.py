@@ -16,6 +16,11 @@ for that computation.
 
 The compute step is `partial`.  On the GPU it is ra_attn_partial: the library's kernels, fp32
 accumulator, LSE merge in its epilogue.  The CPU tests of this module pass an oracle-backed step.
+
+`stage_through_host=True` moves each K/V shard through pinned host memory instead of sending the
+device tensors: for process groups whose backend has no device point-to-point (gloo), and for
+ranks that share one GPU, whose kernels must never wait on one another.  The device-side work of
+every step is the same.
 """
 
 from __future__ import annotations
@@ -42,7 +47,7 @@ def _peer(group, group_rank: int) -> int:
 
 
 def ring_attention_dist(q, k, v, layout: str = "contiguous", causal: bool = True, scale: float = 0.0,
-                        group=None, partial=None):
+                        group=None, partial=None, stage_through_host: bool = False):
     """Ring attention of this rank's shards.
 
     q: [B, H, n_local, d], this rank's query shard; k, v: [B, H_kv, n_local, d], the K/V shard that
@@ -52,6 +57,7 @@ def ring_attention_dist(q, k, v, layout: str = "contiguous", causal: bool = True
     rows over the whole sequence.  Rows with no visible key get O = 0, LSE = -inf.
     partial(q, k, v, o_acc, lse_acc, q_pos, kv_pos, causal, scale, accumulate): one ring step,
     defaulting to the library's ra_attn_partial.
+    stage_through_host: send and receive host copies of the shards (see the module docstring).
     """
     P = dist.get_world_size(group)
     r = dist.get_rank(group)
@@ -68,17 +74,33 @@ def ring_attention_dist(q, k, v, layout: str = "contiguous", causal: bool = True
     k_cur, v_cur = k.contiguous(), v.contiguous()
     k_nxt, v_nxt = torch.empty_like(k_cur), torch.empty_like(v_cur)
     to_next, from_prev = _peer(group, (r + 1) % P), _peer(group, (r - 1) % P)
+    staged = stage_through_host and k_cur.device.type != "cpu"
+    if staged:
+        pin = torch.cuda.is_available()
+        host = [torch.empty(k_cur.shape, dtype=k_cur.dtype, pin_memory=pin) for _ in range(4)]
     for t in range(P):
         reqs = []
         if t + 1 < P:
-            ops = [dist.P2POp(dist.isend, k_cur, to_next, group), dist.P2POp(dist.irecv, k_nxt, from_prev, group),
-                   dist.P2POp(dist.isend, v_cur, to_next, group), dist.P2POp(dist.irecv, v_nxt, from_prev, group)]
+            if staged:
+                # The shard held now goes out from a host copy; the next one arrives in host memory.
+                host[0].copy_(k_cur)
+                host[1].copy_(v_cur)
+                bufs = (host[0], host[2], host[1], host[3])
+            else:
+                bufs = (k_cur, k_nxt, v_cur, v_nxt)
+            ops = [dist.P2POp(dist.isend, bufs[0], to_next, group), dist.P2POp(dist.irecv, bufs[1], from_prev, group),
+                   dist.P2POp(dist.isend, bufs[2], to_next, group), dist.P2POp(dist.irecv, bufs[3], from_prev, group)]
             reqs = dist.batch_isend_irecv(ops)
         s = (r - t) % P  # the K/V shard held at step t
         partial(q, k_cur, v_cur, o_acc, lse_acc, q_pos, shard_positions(layout, P, s, n_local), causal, scale,
                 t > 0)
         for req in reqs:
             req.wait()
+        if staged and t + 1 < P:
+            # Ordered on the current stream after this step's partial, which reads the other buffer.
+            k_nxt.copy_(host[2], non_blocking=True)
+            v_nxt.copy_(host[3], non_blocking=True)
+            torch.cuda.current_stream(k_nxt.device).synchronize()  # the host buffers are reused next step
         k_cur, k_nxt = k_nxt, k_cur
         v_cur, v_nxt = v_nxt, v_cur
     return o_acc, lse_acc

@@ -92,7 +92,7 @@ def test_ring_over_gloo_ranks_matches_the_oracle(world, layout, causal, H, H_kv)
     import torch.multiprocessing as mp
 
     port = _free_port()
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()
     out = manager.dict()
     mp.start_processes(_worker, args=(world, port, layout, causal, H, H_kv, out), nprocs=world,
                        start_method="spawn", join=True)
