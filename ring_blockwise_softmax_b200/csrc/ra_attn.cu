@@ -168,6 +168,11 @@ ra_status_t check_head_dim(int d, int dtype) {
 
 int padded_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : 128); }
 
+// Rows of one K/V tile of the tensor-core forward kernel (the TMA box height of K and V).
+int kv_box_rows(int dp) {
+  return dp == 32 ? ra::FmhaCfg<32>::BN : (dp == 64 ? ra::FmhaCfg<64>::BN : ra::FmhaCfg<128>::BN);
+}
+
 float resolve_scale(float scale, int d) { return scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt((double)d)); }
 
 // ------------------------------------------------------------------------------------------
@@ -501,8 +506,8 @@ static ra_status_t attn_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, con
   if (q->dtype == RA_BF16) {
     const int dp = padded_dim(w.d);
     if ((st = encode_view(&maps.q, shard_view(q, w.n_q, 1, 0, 1), dp)) != RA_OK) return st;
-    if ((st = encode_view(&maps.k, shard_view(k, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
-    if ((st = encode_view(&maps.v, shard_view(v, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.k, shard_view(k, w.n_kv, 1, 0, 1), dp, kv_box_rows(dp))) != RA_OK) return st;
+    if ((st = encode_view(&maps.v, shard_view(v, w.n_kv, 1, 0, 1), dp, kv_box_rows(dp))) != RA_OK) return st;
   }
   st = launch_attention(q, &maps, w, 1, ra::kEpiOut, dev.sms, reinterpret_cast<cudaStream_t>(stream));
   return st == RA_OK ? ok() : st;
@@ -546,8 +551,8 @@ ra_status_t ra_attn_partial(const ra_tensor_t* q, const ra_tensor_t* k_shard, co
   if (q->dtype == RA_BF16) {
     const int dp = padded_dim(w.d);
     if ((st = encode_view(&maps.q, shard_view(q, w.n_q, 1, 0, 1), dp)) != RA_OK) return st;
-    if ((st = encode_view(&maps.k, shard_view(k_shard, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
-    if ((st = encode_view(&maps.v, shard_view(v_shard, w.n_kv, 1, 0, 1), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.k, shard_view(k_shard, w.n_kv, 1, 0, 1), dp, kv_box_rows(dp))) != RA_OK) return st;
+    if ((st = encode_view(&maps.v, shard_view(v_shard, w.n_kv, 1, 0, 1), dp, kv_box_rows(dp))) != RA_OK) return st;
   }
   st = launch_attention(q, &maps, w, 1, accumulate ? ra::kEpiAcc : ra::kEpiPart, dev.sms,
                         reinterpret_cast<cudaStream_t>(stream));
@@ -723,8 +728,8 @@ static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, con
   if (q->dtype == RA_BF16) {
     const int dp = padded_dim(w.d);
     if ((st = encode_view(&maps.q, shard_view(q, n_local, P, shard_rows, tok_rows), dp)) != RA_OK) return st;
-    if ((st = encode_view(&maps.k, shard_view(k, n_local, P, shard_rows, tok_rows), dp)) != RA_OK) return st;
-    if ((st = encode_view(&maps.v, shard_view(v, n_local, P, shard_rows, tok_rows), dp)) != RA_OK) return st;
+    if ((st = encode_view(&maps.k, shard_view(k, n_local, P, shard_rows, tok_rows), dp, kv_box_rows(dp))) != RA_OK) return st;
+    if ((st = encode_view(&maps.v, shard_view(v, n_local, P, shard_rows, tok_rows), dp, kv_box_rows(dp))) != RA_OK) return st;
   }
 
   // Every launch of the call is described and checked before the first one is enqueued.

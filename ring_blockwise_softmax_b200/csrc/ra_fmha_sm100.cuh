@@ -43,31 +43,43 @@
 
 namespace ra {
 
+#ifndef RA_D128_BN64
+#define RA_D128_BN64 1
+#endif
+
 template <int DP>
 struct FmhaCfg {
   static_assert(DP == 32 || DP == 64 || DP == 128, "padded head dim must be 32, 64 or 128");
   static constexpr int BM = 128;    // rows of one query tile
-  static constexpr int BN = 128;    // keys of one K/V tile
+  // Keys of one K/V tile.  At DP = 128 the two O accumulators take half of tensor memory, so
+  // 64-key tiles are what leaves room for S and P in separate columns (see P_SEP).
+  static constexpr int BN = (DP == 128 && RA_D128_BN64) ? 64 : 128;
   static constexpr int ROWS = 256;  // query rows of one work item (two tiles)
   static constexpr int CB = (DP == 32) ? 32 : 64;  // columns per TMA box / swizzle span
   static constexpr int NCB = DP / CB;
   static constexpr int ROW_BYTES = CB * 2;
   static constexpr uint32_t SWZ = (DP == 32) ? kSwizzle64B : kSwizzle128B;
   static constexpr int ATOM_BYTES = 8 * ROW_BYTES;
-  static constexpr int BLOCK_BYTES = 128 * ROW_BYTES;
-  static constexpr int TILE_BYTES = 128 * DP * 2;
-  static constexpr int STAGES = (DP == 128) ? 2 : (DP == 64 ? 5 : 8);
-  static constexpr bool P_SEP = DP <= 64;
-  // P in its own columns: one MMA issuer per query tile.  P over S: one issuer in a fixed
-  // PV_0, QK_0, PV_1, QK_1 order, which staggers the two tiles on the tensor core.
+  static constexpr int Q_BLOCK_BYTES = BM * ROW_BYTES;   // one CB-column block of a Q tile
+  static constexpr int KV_BLOCK_BYTES = BN * ROW_BYTES;  // one CB-column block of a K or V tile
+  static constexpr int Q_TILE_BYTES = BM * DP * 2;
+  static constexpr int KV_TILE_BYTES = BN * DP * 2;
+  static constexpr int STAGES = (DP == 128) ? (BN == 64 ? 4 : 2) : (DP == 64 ? 5 : 8);
+  // P in its own tensor-memory columns, so S_q may be overwritten as soon as the softmax holds it
+  // in registers: one MMA issuer per query tile.  P over S (DP = 128 with 128-key tiles): one
+  // issuer in a fixed PV_0, QK_0, PV_1, QK_1 order, which staggers the two tiles.
+  static constexpr bool P_SEP = DP <= 64 || BN == 64;
   static constexpr int ISSUERS = P_SEP ? 2 : 1;
   static constexpr int S_COL0 = 0;
+  static constexpr int S_STRIDE = BN;
   static constexpr int O_COL0 = 256;
   static constexpr int O_STRIDE = (DP == 128) ? 128 : 64;
-  static constexpr int P_COL0 = P_SEP ? 384 : 0;
-  static constexpr int P_STRIDE = P_SEP ? 64 : 128;
-  static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * STAGES);
-  static constexpr int NBAR = 3 + 3 * STAGES + 9 * 2;
+  static constexpr int P_COL0 = P_SEP ? (DP == 128 ? 2 * BN : 384) : 0;
+  static constexpr int P_STRIDE = P_SEP ? BN / 2 : 128;
+  static_assert(!P_SEP || P_COL0 + 2 * P_STRIDE <= (DP == 128 ? O_COL0 : 512), "tensor memory columns overlap");
+  static constexpr int NSC = BN / 32;  // 32-column chunks of one S row
+  static constexpr int SMEM_TILES = 2 * Q_TILE_BYTES + 2 * STAGES * KV_TILE_BYTES;
+  static constexpr int NBAR = 3 + 3 * STAGES + 10 * 2;
   static constexpr int STATS_BYTES = 2 * 128 * 8;
   static constexpr int PLAN_BYTES = 2 * 64;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES + PLAN_BYTES;
@@ -90,6 +102,17 @@ struct RegSplit {
 #define RA_EMU_EVERY 0
 #endif
 constexpr int kEmuEvery = RA_EMU_EVERY;  // 1 in kEmuEvery column pairs of unmasked tiles use the FMA-pipe exp2
+
+#ifndef RA_EXP_ALTERNATE
+#define RA_EXP_ALTERNATE 1
+#endif
+// The two softmax warpgroups take turns at their exponential loops (see the softmax role).  With
+// 64-key tiles (DP = 128) one warpgroup's exponentials take less time than its per-tile hand-offs,
+// so the turns hide them (measured +2-4 %); with 128-key tiles (DP <= 64) they lose 10-15 %.
+template <int DP>
+constexpr bool alternate_exps() {
+  return RA_EXP_ALTERNATE != 0 && FmhaCfg<DP>::BN == 64;
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -303,7 +326,7 @@ struct Walk {
 // causal bound), start from its first row (the sliding-window bound; 0 without a window).  The
 // walk covers the 128-key tiles that meet that range.  WIN: the launch has a sliding window
 // (compiled separately so that the plain path carries none of its arithmetic).
-template <bool WIN>
+template <bool WIN, int BN>
 __device__ __forceinline__ bool walk_seek(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
   for (; k.step < n_steps; ++k.step) {
     const int s = ring_shard(w, it.r, w.ring_step + k.step);
@@ -312,37 +335,37 @@ __device__ __forceinline__ bool walk_seek(Walk& k, const AttnWork& w, const Item
     if (lim > start) {
       k.s = s;
       k.lim = lim;
-      k.u0 = start & ~(FmhaCfg<32>::BN - 1);
+      k.u0 = start & ~(BN - 1);
       return true;
     }
   }
   return false;
 }
 
-template <bool WIN>
+template <bool WIN, int BN>
 __device__ __forceinline__ bool walk_begin(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
   k.step = 0;
-  return walk_seek<WIN>(k, w, it, n_steps);
+  return walk_seek<WIN, BN>(k, w, it, n_steps);
 }
 
-template <bool WIN>
+template <bool WIN, int BN>
 __device__ __forceinline__ bool walk_next(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
-  k.u0 += FmhaCfg<32>::BN;
+  k.u0 += BN;
   if (k.u0 < k.lim) return true;
   ++k.step;
-  return walk_seek<WIN>(k, w, it, n_steps);
+  return walk_seek<WIN, BN>(k, w, it, n_steps);
 }
 
 
 // Number of K/V tiles the item walks (what the MMA issuer needs; it never reads the keys).
-template <bool WIN>
+template <bool WIN, int BN>
 __device__ __forceinline__ int walk_count(const AttnWork& w, const Item& it, int n_steps) {
   int n = 0;
   for (int step = 0; step < n_steps; ++step) {
     const int s = ring_shard(w, it.r, w.ring_step + step);
     const int lim = visible_key_limit(w, it.pos_last, s);
     const int start = WIN ? visible_key_start(w, it.pos_first, s) : 0;
-    if (lim > start) n += (lim + FmhaCfg<32>::BN - 1) / FmhaCfg<32>::BN - start / FmhaCfg<32>::BN;
+    if (lim > start) n += (lim + BN - 1) / BN - start / BN;
   }
   return n;
 }
@@ -358,7 +381,7 @@ struct DescBase {
   uint64_t vmn;   // MN-major V: leading = next 64-column block, stride = one 8-row swizzle atom
   __device__ __forceinline__ DescBase() {
     kmaj = make_smem_desc(0, 16, C::ATOM_BYTES, C::SWZ);
-    vmn = make_smem_desc(0, C::BLOCK_BYTES, C::ATOM_BYTES, C::SWZ);
+    vmn = make_smem_desc(0, C::KV_BLOCK_BYTES, C::ATOM_BYTES, C::SWZ);
   }
 };
 
@@ -375,13 +398,14 @@ __device__ __forceinline__ void fmha_issue_qk(const DescBase<C>& db, uint32_t d_
 #pragma unroll
   for (int kk = 0; kk < C::D / 16; ++kk) {
     const int cb = (kk * 16) / C::CB;
-    const uint32_t off = (cb * C::BLOCK_BYTES + ((kk * 16) % C::CB) * 2) >> 4;  // compile-time
-    mma_ss(d_s, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+    const uint32_t off_a = (cb * C::Q_BLOCK_BYTES + ((kk * 16) % C::CB) * 2) >> 4;  // compile-time
+    const uint32_t off_b = (cb * C::KV_BLOCK_BYTES + ((kk * 16) % C::CB) * 2) >> 4;
+    mma_ss(d_s, a0 + off_a, b0 + off_b, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 // O[tmem d_o] (+)= P (bf16 pairs in tensor memory at p_tmem) * V (MN-major at v_addr): 16 keys
-// per MMA; the next 64-column block of V sits one BLOCK_BYTES further (leading byte offset).
+// per MMA; the next 64-column block of V sits one KV_BLOCK_BYTES further (leading byte offset).
 template <class C>
 __device__ __forceinline__ void fmha_issue_pv(const DescBase<C>& db, uint32_t d_o, uint32_t p_tmem, uint32_t v_addr,
                                               uint32_t idesc, bool accumulate) {
@@ -478,9 +502,9 @@ __device__ __forceinline__ void fmha_epilogue_row(const AttnWork& w, const Item&
 // bf16 pairs in pk (the row of P_q); row sums accumulated in two packed fp32x2 chains.  EVERY > 0: one column pair in
 // EVERY goes to the FMA-pipe polynomial instead of the MUFU (only for tiles without masked
 // scores, see exp2_poly3).
-template <int EVERY, int E0 = 0, int E1 = 64>
-__device__ __forceinline__ void softmax_exp(const uint32_t (&sr)[4][32], float sl2, float base, uint32_t (&pk)[64],
-                                            float2 (&rs)[2]) {
+template <int EVERY, int E0, int E1, int NSC>
+__device__ __forceinline__ void softmax_exp(const uint32_t (&sr)[NSC][32], float sl2, float base,
+                                            uint32_t (&pk)[NSC * 16], float2 (&rs)[2]) {
   const float2 sc = make_float2(sl2, sl2);
   const float2 nb = make_float2(-base, -base);
 #pragma unroll
@@ -501,13 +525,13 @@ __device__ __forceinline__ void softmax_exp(const uint32_t (&sr)[4][32], float s
 
 // As softmax_exp, but each 16-pair chunk of P_q goes to tensor memory as soon as it is computed
 // (fewer live registers; used where P_q's columns are known to be free before the exponentials).
-template <int EVERY>
-__device__ __forceinline__ void softmax_exp_store(const uint32_t (&sr)[4][32], float sl2, float base, uint32_t p_addr,
-                                                  float2 (&rs)[2]) {
+template <int EVERY, int NSC>
+__device__ __forceinline__ void softmax_exp_store(const uint32_t (&sr)[NSC][32], float sl2, float base,
+                                                  uint32_t p_addr, float2 (&rs)[2]) {
   const float2 sc = make_float2(sl2, sl2);
   const float2 nb = make_float2(-base, -base);
 #pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {
+  for (int cc = 0; cc < NSC; ++cc) {
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -539,9 +563,9 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
 
   uint8_t* sQ = smem;  // two tiles
-  uint8_t* sK = sQ + 2 * C::TILE_BYTES;
-  uint8_t* sV = sK + C::STAGES * C::TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + C::STAGES * C::TILE_BYTES);
+  uint8_t* sK = sQ + 2 * C::Q_TILE_BYTES;
+  uint8_t* sV = sK + C::STAGES * C::KV_TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + C::STAGES * C::KV_TILE_BYTES);
   uint64_t* bar_q_full = bars;
   uint64_t* bar_q_empty = bars + 1;
   uint64_t* bar_mma_done = bars + 2;
@@ -557,7 +581,8 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_s_free = bar_stats + 2;             // [2] softmax has loaded S_q into registers
   uint64_t* bar_plan_full = bar_s_free + 2;         // [2] item plan slot written
   uint64_t* bar_plan_empty = bar_plan_full + 2;     // [2] item plan slot read by every consumer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_plan_empty + 2);
+  uint64_t* bar_exp_done = bar_plan_empty + 2;      // [2] softmax warpgroup q finished an exponential phase
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_exp_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* stats = reinterpret_cast<float2*>(tmem_slot + 4);  // [2][128] (m_used, l_sum)
   ItemPlan* plan = reinterpret_cast<ItemPlan*>(stats + 2 * 128);  // [2], slot = item sequence & 1
@@ -586,6 +611,7 @@ __global__ void __launch_bounds__(512, 1)
       // Readers of a plan slot (d <= 64): each MMA issuer thread, 8 softmax warps, 4 epilogue warps.
       mbar_init(bar_plan_full + q, 1);
       mbar_init(bar_plan_empty + q, C::ISSUERS + 12);
+      mbar_init(bar_exp_done + q, 4);  // one arrival per softmax warp
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -622,38 +648,38 @@ __global__ void __launch_bounds__(512, 1)
           const int slot = it_seq & 1;
           if (it_seq >= 2 && !mbar_wait(bar_plan_empty + slot, ((it_seq >> 1) - 1) & 1, ctl, 0x103)) break;
           plan[slot].it = it;
-          plan[slot].n = walk_count<WIN>(w, it, n_steps);
+          plan[slot].n = walk_count<WIN, C::BN>(w, it, n_steps);
           mbar_arrive(bar_plan_full + slot);
           ++it_seq;
         }
         Walk wk;
-        bool has = walk_begin<WIN>(wk, w, it, n_steps);
+        bool has = walk_begin<WIN, C::BN>(wk, w, it, n_steps);
         if (!has) continue;
         if (it_q > 0 && !mbar_wait(bar_q_empty, (it_q - 1) & 1, ctl, 0x101)) break;
-        mbar_arrive_expect_tx(bar_q_full, 2 * C::TILE_BYTES);
+        mbar_arrive_expect_tx(bar_q_full, 2 * C::Q_TILE_BYTES);
 #pragma unroll
         for (int q = 0; q < 2; ++q)
 #pragma unroll
           for (int cb = 0; cb < C::NCB; ++cb)
-            tma_load_5d(sQ + q * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_q, bar_q_full, cb * C::CB,
+            tma_load_5d(sQ + q * C::Q_TILE_BYTES + cb * C::Q_BLOCK_BYTES, &tm_q, bar_q_full, cb * C::CB,
                         it.t0 + 128 * q, it.r, it.h, it.b);
         ++it_q;
-        for (; has; has = walk_next<WIN>(wk, w, it, n_steps)) {
+        for (; has; has = walk_next<WIN, C::BN>(wk, w, it, n_steps)) {
           const int st = static_cast<int>(g % C::STAGES);
           if (g >= C::STAGES &&
               !mbar_wait(bar_kv_empty + st, static_cast<uint32_t>((g / C::STAGES) - 1) & 1, ctl, 0x102)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar_k_full + st, C::TILE_BYTES);
+          mbar_arrive_expect_tx(bar_k_full + st, C::KV_TILE_BYTES);
 #pragma unroll
           for (int cb = 0; cb < C::NCB; ++cb)
-            tma_load_5d(sK + st * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_k, bar_k_full + st, cb * C::CB, wk.u0,
+            tma_load_5d(sK + st * C::KV_TILE_BYTES + cb * C::KV_BLOCK_BYTES, &tm_k, bar_k_full + st, cb * C::CB, wk.u0,
                         wk.s, it.hk, it.b);
-          mbar_arrive_expect_tx(bar_v_full + st, C::TILE_BYTES);
+          mbar_arrive_expect_tx(bar_v_full + st, C::KV_TILE_BYTES);
 #pragma unroll
           for (int cb = 0; cb < C::NCB; ++cb)
-            tma_load_5d(sV + st * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tm_v, bar_v_full + st, cb * C::CB, wk.u0,
+            tma_load_5d(sV + st * C::KV_TILE_BYTES + cb * C::KV_BLOCK_BYTES, &tm_v, bar_v_full + st, cb * C::CB, wk.u0,
                         wk.s, it.hk, it.b);
           ++g;
         }
@@ -685,7 +711,7 @@ __global__ void __launch_bounds__(512, 1)
         if (idx >= n_items) continue;
         Item it;
         decode_item(w, idx, it);
-        const int n = walk_count<WIN>(w, it, n_steps);
+        const int n = walk_count<WIN, C::BN>(w, it, n_steps);
         if (n == 0) {
           for (int q = 0; q < 2 && ok && it_all > 0; ++q)
             ok = mbar_wait_issuer(bar_o_empty + q, (it_all - 1) & 1, ctl, 0x208);
@@ -700,8 +726,8 @@ __global__ void __launch_bounds__(512, 1)
         for (int q = 0; q < 2 && ok; ++q) {
           if (g > 0 && !(ok = mbar_wait_issuer(bar_pv_done + q, static_cast<uint32_t>(g - 1) & 1, ctl, 0x203))) break;
           tc_fence_after();
-          fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
-                           k_base + static_cast<int>(g % C::STAGES) * C::TILE_BYTES, idesc_qk);
+          fmha_issue_qk<C>(db, tmem + C::S_COL0 + C::S_STRIDE * q, q_base + q * C::Q_TILE_BYTES,
+                           k_base + static_cast<int>(g % C::STAGES) * C::KV_TILE_BYTES, idesc_qk);
           mma_commit(bar_s_full + q);
         }
         if (!ok) break;
@@ -716,7 +742,7 @@ __global__ void __launch_bounds__(512, 1)
             if (!ok) break;
             tc_fence_after();
             fmha_issue_pv<C>(db, tmem + C::O_COL0 + C::O_STRIDE * q, tmem + C::P_COL0 + C::P_STRIDE * q,
-                             v_base + static_cast<int>(gj % C::STAGES) * C::TILE_BYTES, idesc_pv, j > 0);
+                             v_base + static_cast<int>(gj % C::STAGES) * C::KV_TILE_BYTES, idesc_pv, j > 0);
             mma_commit(bar_pv_done + q);
             if (has_next) {
               const long long gn = gj + 1;
@@ -725,8 +751,8 @@ __global__ void __launch_bounds__(512, 1)
                                         static_cast<uint32_t>(gn / C::STAGES) & 1, nullptr, 0, ctl, 0x209);
               if (!ok) break;
               tc_fence_after();
-              fmha_issue_qk<C>(db, tmem + C::S_COL0 + 128 * q, q_base + q * C::TILE_BYTES,
-                               k_base + static_cast<int>(gn % C::STAGES) * C::TILE_BYTES, idesc_qk);
+              fmha_issue_qk<C>(db, tmem + C::S_COL0 + C::S_STRIDE * q, q_base + q * C::Q_TILE_BYTES,
+                               k_base + static_cast<int>(gn % C::STAGES) * C::KV_TILE_BYTES, idesc_qk);
               mma_commit(bar_s_full + q);
               if (q == 1 && j + 2 == n) mma_commit(bar_q_empty);  // last QKs of the item issued
             }
@@ -759,10 +785,10 @@ __global__ void __launch_bounds__(512, 1)
       const int q = warp - 13;
       constexpr uint32_t idesc_qk = make_idesc_bf16(128, C::BN, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, DP, 0, 1);
-      const uint32_t q_addr = smem_addr(sQ) + q * C::TILE_BYTES;
+      const uint32_t q_addr = smem_addr(sQ) + q * C::Q_TILE_BYTES;
       const uint32_t k_base = smem_addr(sK);
       const uint32_t v_base = smem_addr(sV);
-      const uint32_t d_s = tmem + C::S_COL0 + 128 * q;
+      const uint32_t d_s = tmem + C::S_COL0 + C::S_STRIDE * q;
       const uint32_t d_o = tmem + C::O_COL0 + C::O_STRIDE * q;
       const uint32_t p_t = tmem + C::P_COL0 + C::P_STRIDE * q;
       const DescBase<C> db;
@@ -778,7 +804,7 @@ __global__ void __launch_bounds__(512, 1)
                                   ctl, 0x202))
           return false;
         tc_fence_after();
-        fmha_issue_qk<C>(db, d_s, q_addr, k_base + static_cast<int>(gk % C::STAGES) * C::TILE_BYTES, idesc_qk);
+        fmha_issue_qk<C>(db, d_s, q_addr, k_base + static_cast<int>(gk % C::STAGES) * C::KV_TILE_BYTES, idesc_qk);
         mma_commit(bar_s_full + q);
         ++cq;
         if (last_of_item) mma_commit(bar_q_empty);
@@ -800,7 +826,7 @@ __global__ void __launch_bounds__(512, 1)
                                       (j > 0 || it_all == 0) ? nullptr : bar_o_empty + q, (it_all - 1) & 1, ctl, 0x206);
             if (!ok) break;
             tc_fence_after();
-            fmha_issue_pv<C>(db, d_o, p_t, v_base + static_cast<int>(gj % C::STAGES) * C::TILE_BYTES, idesc_pv,
+            fmha_issue_pv<C>(db, d_o, p_t, v_base + static_cast<int>(gj % C::STAGES) * C::KV_TILE_BYTES, idesc_pv,
                              j > 0);
             mma_commit(bar_pv_done + q);
             ++cpv;
@@ -828,7 +854,7 @@ __global__ void __launch_bounds__(512, 1)
     const int q = warp >> 2;
     const int row = threadIdx.x & 127;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t s_addr = lane_addr + C::S_COL0 + 128 * q;
+    const uint32_t s_addr = lane_addr + C::S_COL0 + C::S_STRIDE * q;
     const uint32_t p_addr = lane_addr + C::P_COL0 + C::P_STRIDE * q;
     const uint32_t o_addr = lane_addr + C::O_COL0 + C::O_STRIDE * q;
     const float sl2 = w.scale_log2;
@@ -856,7 +882,7 @@ __global__ void __launch_bounds__(512, 1)
       float l_sum = 0.f;         // running sum of 2^(x - m_used)
       Walk wk;
       int cur_s = -1, row_lim = 0, row_lo = 0;
-      for (bool has = walk_begin<WIN>(wk, w, it, n_steps); has; has = walk_next<WIN>(wk, w, it, n_steps)) {
+      for (bool has = walk_begin<WIN, C::BN>(wk, w, it, n_steps); has; has = walk_next<WIN, C::BN>(wk, w, it, n_steps)) {
         if (wk.s != cur_s) {
           cur_s = wk.s;
           row_lim = row_ok ? visible_key_limit(w, pos_q, wk.s) : w.n_kv;
@@ -868,13 +894,13 @@ __global__ void __launch_bounds__(512, 1)
         }
         s_seen = false;
         tc_fence_after();
-        uint32_t sr[4][32];
+        constexpr int NSC = C::NSC;
+        uint32_t sr[NSC][32];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_addr + cc * 32, sr[cc]);
+        for (int cc = 0; cc < NSC; ++cc) tmem_ld32(s_addr + cc * 32, sr[cc]);
         tmem_ld_wait(sr[0]);
-        reg_dep(sr[1]);
-        reg_dep(sr[2]);
-        reg_dep(sr[3]);
+#pragma unroll
+        for (int cc = 1; cc < NSC; ++cc) reg_dep(sr[cc]);
         if (C::P_SEP) {
           // S_q is in registers: the next QK_q may overwrite it while this tile's softmax runs.
           tc_fence_before();
@@ -886,16 +912,16 @@ __global__ void __launch_bounds__(512, 1)
         const bool masked = __any_sync(0xffffffffu, cut);
         if (cut) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e)
+          for (int e = 0; e < C::BN; ++e)
             if (e >= lim || (WIN && e < lo)) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
         }
-        // Row max as 8 independent chains (a single chain of 128 dependent max operations would
+        // Row max as 8 independent chains (a single chain of BN dependent max operations would
         // be latency-bound).
         float mxp[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mxp[i] = __uint_as_float(sr[0][i]);
 #pragma unroll
-        for (int e = 8; e < 128; e += 2)
+        for (int e = 8; e < C::BN; e += 2)
           mxp[(e >> 1) & 7] = fmax3(mxp[(e >> 1) & 7], __uint_as_float(sr[e >> 5][e & 31]),
                                     __uint_as_float(sr[(e + 1) >> 5][(e + 1) & 31]));
         const float mx = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
@@ -919,16 +945,31 @@ __global__ void __launch_bounds__(512, 1)
           // P_q has its own columns, which the previous PV_q may still be reading.  The
           // exponentials are computed into registers first, so by the time of this wait that PV
           // has almost always landed.
-          uint32_t pk[64];
+          constexpr int HALF = NSC * 8;  // column pairs in half a row
+          uint32_t pk[NSC * 16];
           bool pv_seen;
+          if (alternate_exps<DP>()) {
+            // Exponential phases alternate between the two warpgroups: tile c of warpgroup 0
+            // waits for phase c - 1 of warpgroup 1, which waits for phase c of warpgroup 0.
+            const bool first = q == 0 && c == 0;
+            if (!first) {
+              const uint32_t par = q == 0 ? static_cast<uint32_t>(c - 1) & 1 : static_cast<uint32_t>(c) & 1;
+              ok = __all_sync(0xffffffffu, mbar_wait(bar_exp_done + (q ^ 1), par, ctl, 0x306));
+              if (!ok) break;
+            }
+          }
           if (masked || kEmuEvery == 0) {
-            softmax_exp<0, 0, 32>(sr, sl2, base, pk, rsp);
+            softmax_exp<0, 0, HALF>(sr, sl2, base, pk, rsp);
             pv_seen = c == 0 || mbar_test_wait(bar_pv_done + q, (c - 1) & 1);
-            softmax_exp<0, 32, 64>(sr, sl2, base, pk, rsp);
+            softmax_exp<0, HALF, 2 * HALF>(sr, sl2, base, pk, rsp);
           } else {
-            softmax_exp<kEmuEvery, 0, 32>(sr, sl2, base, pk, rsp);
+            softmax_exp<kEmuEvery, 0, HALF>(sr, sl2, base, pk, rsp);
             pv_seen = c == 0 || mbar_test_wait(bar_pv_done + q, (c - 1) & 1);
-            softmax_exp<kEmuEvery, 32, 64>(sr, sl2, base, pk, rsp);
+            softmax_exp<kEmuEvery, HALF, 2 * HALF>(sr, sl2, base, pk, rsp);
+          }
+          if (alternate_exps<DP>()) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_exp_done + q);
           }
           s_seen = mbar_test_wait(bar_s_full + q, (c + 1) & 1);  // the next QK_q, issued at s_free
           if (!__all_sync(0xffffffffu, pv_seen)) {
@@ -936,7 +977,10 @@ __global__ void __launch_bounds__(512, 1)
             if (!ok) break;
           }
           tc_fence_after();
-          tmem_st64(p_addr, pk);
+          if constexpr (NSC == 4)
+            tmem_st64(p_addr, pk);
+          else
+            tmem_st32(p_addr, pk);
         } else {
           // P_q over S_q: those columns are free once S_q is loaded (the next QK_q waits for this
           // PV_q); only the O rescale needs the previous PV_q to have landed.
@@ -946,9 +990,9 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
           }
           if (masked || kEmuEvery == 0)
-            softmax_exp_store<0>(sr, sl2, base, p_addr, rsp);
+            softmax_exp_store<0, NSC>(sr, sl2, base, p_addr, rsp);
           else
-            softmax_exp_store<kEmuEvery>(sr, sl2, base, p_addr, rsp);
+            softmax_exp_store<kEmuEvery, NSC>(sr, sl2, base, p_addr, rsp);
         }
         if (any_rescale) {
 #pragma unroll
@@ -1005,7 +1049,7 @@ __global__ void __launch_bounds__(512, 1)
       } else {
         decode_item(w, idx, it);
         Walk wk;
-        has_o = walk_begin<WIN>(wk, w, it, n_steps);
+        has_o = walk_begin<WIN, C::BN>(wk, w, it, n_steps);
       }
       for (int q = 0; q < 2; ++q) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_full + q, it_all & 1, ctl, 0x401) &&
