@@ -110,9 +110,9 @@ constexpr int kEmuEvery = RA_EMU_EVERY;  // 1 in kEmuEvery column pairs of unmas
 // 64-key tiles (DP = 128) one warpgroup's exponentials take less time than its per-tile hand-offs,
 // so the turns hide them (measured +2-4 %); with 128-key tiles (DP <= 64) they lose 10-15 %.
 template <int DP>
-constexpr bool alternate_exps() {
-  return RA_EXP_ALTERNATE != 0 && FmhaCfg<DP>::BN == 64;
-}
+struct AlternateExps {
+  static constexpr bool value = RA_EXP_ALTERNATE != 0 && FmhaCfg<DP>::BN == 64;
+};
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -948,7 +948,7 @@ __global__ void __launch_bounds__(512, 1)
           constexpr int HALF = NSC * 8;  // column pairs in half a row
           uint32_t pk[NSC * 16];
           bool pv_seen;
-          if (alternate_exps<DP>()) {
+          if (AlternateExps<DP>::value) {
             // Exponential phases alternate between the two warpgroups: tile c of warpgroup 0
             // waits for phase c - 1 of warpgroup 1, which waits for phase c of warpgroup 0.
             const bool first = q == 0 && c == 0;
@@ -967,7 +967,7 @@ __global__ void __launch_bounds__(512, 1)
             pv_seen = c == 0 || mbar_test_wait(bar_pv_done + q, (c - 1) & 1);
             softmax_exp<kEmuEvery, HALF, 2 * HALF>(sr, sl2, base, pk, rsp);
           }
-          if (alternate_exps<DP>()) {
+          if (AlternateExps<DP>::value) {
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_exp_done + q);
           }
