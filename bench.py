@@ -35,7 +35,7 @@ SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-FMHA_SOURCES = ("ra_common.cuh", "ra_fmha_sm100.cuh", "ra_fmha_launch.cu")
+FMHA_SOURCES = ("ra_common.cuh", "ra_fmha_sm100.cuh", "ra_fmha_launch.cu", "ra_attn.cu")
 
 
 def kernel_sources_hash() -> str:
@@ -329,6 +329,10 @@ def config_dict(w, args):
     name = w.name if w.H_kv is None else f"{w.name}, grouped-query K/V with {w.H_kv} heads"
     if w.window is not None:
         name += f", sliding window of {w.window} positions"
+    from ring_blockwise_softmax_b200 import inputs as I
+
+    if w.N != I.WORKLOADS[w.cfg].N:
+        name += f", sequence length reduced to {w.N}"
     return {"workload": f"cfg{w.cfg}: {name}", "B": w.B, "H": w.H, "H_kv": w.H_kv or w.H, "N": w.N, "d": w.d,
             "causal": w.causal, "window": w.window,
             "P": w.P, "layout": w.layout, "schedule": args.schedule,
@@ -540,7 +544,7 @@ def run_gpu(args, w):
     # The other bf16 workloads, each timed the same way (the headline keys stay on the main one).
     others = {}
     if not args.backward and args.configs:
-        for c in [int(x) for x in args.configs.split(",") if x.strip()]:
+        for c in [int(x) for x in args.configs.split(",") if x.strip().isdigit()]:
             if c == w.cfg:
                 continue
             wc = I.WORKLOADS[c]
@@ -623,6 +627,8 @@ def main(argv=None):
                     help="causal sliding-window variant of a causal workload (window in positions)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query variant of the workload: K and V with this many heads (must divide H)")
+    ap.add_argument("--n", type=int, default=None,
+                    help="sequence length override: a smaller case of the workload's layout (profiling)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the attention kernel, from an ncu capture of the current kernel")
     args = ap.parse_args(argv)
@@ -631,6 +637,12 @@ def main(argv=None):
     from ring_blockwise_softmax_b200 import inputs as I
 
     w = I.WORKLOADS[args.config]
+    if args.n is not None:
+        import dataclasses
+
+        if args.n < w.P or args.n % w.P != 0:
+            raise SystemExit("--n must be a positive multiple of the workload's P")
+        w = dataclasses.replace(w, N=args.n)
     if args.kv_heads is not None:
         if w.tabular is not None or args.kv_heads < 1 or w.H % args.kv_heads != 0:
             raise SystemExit("--kv-heads must divide H and does not apply to the tabular workload")

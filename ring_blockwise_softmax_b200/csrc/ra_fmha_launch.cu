@@ -16,6 +16,13 @@ static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, cons
   auto kern = fmha_fwd_sm100<RA_FMHA_DP, EPI, WIN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
+  // The warpgroups' setmaxnreg shares must fit in the registers the block is launched with, or a
+  // setmaxnreg.inc would never be granted: refuse the launch if the compiled kernel has fewer.
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs * C::THREADS < RegSplit<RA_FMHA_DP, EPI>::kTotal || attr.maxThreadsPerBlock < C::THREADS)
+    return cudaErrorInvalidConfiguration;
   // Persistent grid: one CTA per SM (at most one per work item of 256 query rows).
   const long long n_items = static_cast<long long>((w.n_q + C::ROWS - 1) / C::ROWS) * w.n_r * w.H * w.B;
   if (n_items > 2147483647LL) return cudaErrorInvalidValue;

@@ -46,6 +46,9 @@ namespace ra {
 #ifndef RA_D128_BN64
 #define RA_D128_BN64 1
 #endif
+#ifndef RA_SOFTMAX_SPLIT
+#define RA_SOFTMAX_SPLIT 0
+#endif
 
 template <int DP>
 struct FmhaCfg {
@@ -78,24 +81,47 @@ struct FmhaCfg {
   static constexpr int P_STRIDE = P_SEP ? BN / 2 : 128;
   static_assert(!P_SEP || P_COL0 + 2 * P_STRIDE <= (DP == 128 ? O_COL0 : 512), "tensor memory columns overlap");
   static constexpr int NSC = BN / 32;  // 32-column chunks of one S row
+  // Column-split softmax: two warpgroups per query tile, each taking half of every S row (and
+  // half of the O columns in rescales and the epilogue), so four softmax warps share each SM
+  // sub-partition instead of two and hide one another's barrier / tensor-memory latencies.  The
+  // halves exchange row maxima per tile and row sums per item through shared memory.  The
+  // epilogue runs in the softmax warps (no registers are left for a separate warpgroup).
+  static constexpr bool SPLIT = RA_SOFTMAX_SPLIT != 0 && P_SEP;
+  static constexpr int HCOLS = SPLIT ? BN / 2 : BN;  // S columns per softmax thread
+  static constexpr int SM_WARPS = SPLIT ? 16 : 8;     // softmax warps
+  static constexpr int PROD_WARP = SPLIT ? 16 : 12;   // TMA producer; MMA issuers follow it
   static constexpr int SMEM_TILES = 2 * Q_TILE_BYTES + 2 * STAGES * KV_TILE_BYTES;
-  static constexpr int NBAR = 3 + 3 * STAGES + 10 * 2;
+  static constexpr int NBAR = 3 + 3 * STAGES + 11 * 2;
   static constexpr int STATS_BYTES = 2 * 128 * 8;
   static constexpr int PLAN_BYTES = 2 * 64;
-  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES + PLAN_BYTES;
-  static constexpr int THREADS = 512;
+  static constexpr int XCH_BYTES = SPLIT ? 2 * (2 * 2 * 2 * 128 * 4) : 0;  // row max and row sum exchange
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + NBAR * 8 + 16 + STATS_BYTES + PLAN_BYTES + XCH_BYTES;
+  static constexpr int THREADS = SPLIT ? 640 : 512;
   static constexpr int D = DP;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
 // Per-thread register budgets after setmaxnreg (softmax, epilogue, producer/MMA warpgroups).  The
 // merging epilogues (accumulate modes) need more registers than the plain output one.
 template <int DP, int EPI>
 struct RegSplit {
+  static constexpr bool kSplit = FmhaCfg<DP>::SPLIT;
   static constexpr bool kAcc = (EPI == 2 || EPI == 3);
-  static constexpr int kProd = 80;
-  static constexpr int kEpi = kAcc ? 80 : (DP <= 64 ? 48 : 64);
-  static constexpr int kSoftmax = ((65536 / 128 - kProd - kEpi) / 2) / 8 * 8;
-  static_assert(2 * 128 * kSoftmax + 128 * kEpi + 128 * kProd <= 65536, "register split exceeds the launch");
+  // Registers per thread at launch: 65536 / threads rounded down to a multiple of 8 (the host
+  // checks the compiled kernel's count against this before launching).
+  static constexpr int kLaunch = (65536 / FmhaCfg<DP>::THREADS) / 8 * 8;
+  // Producer / MMA-issuer warpgroup: 64 registers leave the d <= 64 softmax enough to compile
+  // without spills; at d = 128 (64-key tiles) the softmax needs fewer and the others 80.
+  static constexpr int kProd = kSplit ? 64 : (DP == 128 ? 80 : 64);
+  static constexpr int kEpi = kSplit ? 0 : (kAcc ? 80 : (DP <= 64 ? 48 : 64));
+  static constexpr int kSoftmaxWGs = kSplit ? 4 : 2;
+  static constexpr int kSoftmax =
+      ((kLaunch * FmhaCfg<DP>::THREADS / 128 - kProd - kEpi) / kSoftmaxWGs) / 8 * 8;
+  // Every warpgroup's share, added up, must fit in what the block was launched with, or a
+  // setmaxnreg.inc would wait forever.
+  static_assert(kSoftmaxWGs * 128 * kSoftmax + 128 * kEpi + 128 * kProd <= kLaunch * FmhaCfg<DP>::THREADS,
+                "register split exceeds the launch");
+  static constexpr int kTotal = kSoftmaxWGs * 128 * kSoftmax + 128 * kEpi + 128 * kProd;
 };
 
 #ifndef RA_EMU_EVERY
@@ -184,6 +210,9 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
 #ifndef RA_ISSUER_SPIN
 #define RA_ISSUER_SPIN 1
 #endif
+#ifndef RA_ISSUER_BACKOFF_NS
+#define RA_ISSUER_BACKOFF_NS 0
+#endif
 // Wait used by the single-thread MMA issuers: spin on the non-blocking test (a sleeping try_wait
 // wakes up late, and each issuer hop sits on the critical path of a query tile), bounded like
 // mbar_wait.
@@ -193,8 +222,10 @@ __device__ __forceinline__ bool mbar_wait_issuer(uint64_t* bar, uint32_t parity,
   const uint64_t t0 = globaltimer_ns();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 256; ++i)
+    for (int i = 0; i < 256; ++i) {
       if (mbar_test_wait(bar, parity)) return true;
+      if (RA_ISSUER_BACKOFF_NS > 0) __nanosleep(RA_ISSUER_BACKOFF_NS);
+    }
     if (*ctl.abort) return false;
     if (globaltimer_ns() - t0 > ctl.limit_ns) {
       atomicOr(ctl.status, kDevStatusTimeout);
@@ -212,6 +243,9 @@ __device__ __forceinline__ bool mbar_wait_issuer(uint64_t* bar, uint32_t parity,
 // adding up.  Bounded like mbar_wait.
 __device__ __forceinline__ bool mbar_wait_all_issuer(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
                                                      uint32_t p2, const WaitCtl& ctl, unsigned site) {
+  if (!RA_ISSUER_SPIN)
+    return (b0 == nullptr || mbar_wait(b0, p0, ctl, site)) && (b1 == nullptr || mbar_wait(b1, p1, ctl, site)) &&
+           (b2 == nullptr || mbar_wait(b2, p2, ctl, site));
   bool d0 = b0 == nullptr, d1 = b1 == nullptr, d2 = b2 == nullptr;
   auto poll = [&]() -> bool {
     const bool t0 = d0 || mbar_test_wait(b0, p0);
@@ -220,6 +254,7 @@ __device__ __forceinline__ bool mbar_wait_all_issuer(uint64_t* b0, uint32_t p0, 
     d0 = t0;
     d1 = t1;
     d2 = t2;
+    if (RA_ISSUER_BACKOFF_NS > 0 && !(t0 && t1 && t2)) __nanosleep(RA_ISSUER_BACKOFF_NS);
     return t0 && t1 && t2;
   };
   if (poll()) return true;
@@ -498,6 +533,114 @@ __device__ __forceinline__ void fmha_epilogue_row(const AttnWork& w, const Item&
   }
 }
 
+#ifndef RA_SPLIT_WARP_ARRIVE
+#define RA_SPLIT_WARP_ARRIVE 0
+#endif
+// Column-split softmax: arrivals on the per-tile barriers (S consumed, P written) one per warp
+// instead of one per thread.
+constexpr bool kSplitWarpArrive = RA_SPLIT_WARP_ARRIVE != 0;
+
+// The 8 warps of one query tile's two column-split softmax warpgroups meet on `bar` (an mbarrier
+// counting one arrival per warp, after the warp's own lanes have synchronised; n counts this
+// thread's meetings so far).  Bounded like every wait: returns false if it ran out or the CTA is
+// aborting.
+__device__ __forceinline__ bool pair_meet(uint64_t* bar, int& n, const WaitCtl& ctl) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, static_cast<uint32_t>(n) & 1, ctl, 0x307);
+  ++n;
+  return ok;
+}
+
+// fmha_epilogue_row for the column-split softmax: this thread's half of the row, O columns
+// [half * D/2, (half + 1) * D/2).  Both halves hold the same (m, l); half 0 writes the LSE.  In
+// the in-place accumulate mode the pair meets between reading the stored LSE and overwriting it.
+template <class C, int EPI>
+__device__ __forceinline__ void fmha_epilogue_row_half(const AttnWork& w, const Item& it, int t, bool row_ok,
+                                                       bool has_o, float2 ml, uint32_t o_addr, int half,
+                                                       uint64_t* pair_bar, int& pair_n, const WaitCtl& ctl) {
+  constexpr int HD = C::D / 2;           // O columns of this half
+  constexpr int CH = HD < 32 ? HD : 32;  // columns per tensor-memory load
+  const bool has = ml.y > 0.f;
+  const float inv_l = has ? 1.f / ml.y : 0.f;
+  const float lse_part = has ? (ml.x * 0.69314718055994531f + logf(ml.y)) : -INFINITY;
+  const bool skip = (EPI == kEpiAcc) && !has;  // merging an empty partial is the identity
+  float L = lse_part, w_part = 1.f, w_acc = 0.f;
+  float* acc_row = nullptr;
+  float* accl_ptr = nullptr;
+  if (EPI != kEpiOut) {
+    acc_row = w.acc_o + it.b * w.a_sb + it.h * w.a_sh + it.r * w.a_rs + static_cast<long long>(t) * w.a_ts;
+    accl_ptr = w.acc_l + it.b * w.al_sb + it.h * w.al_sh + it.r * w.al_rs + static_cast<long long>(t) * w.al_ts;
+  }
+  if ((EPI == kEpiAcc || EPI == kEpiAccOut) && row_ok && !skip) {
+    const float la = *accl_ptr;
+    lse_merge_weights(la, lse_part, L, w_acc, w_part);
+  }
+  if (EPI == kEpiAcc) (void)pair_meet(pair_bar, pair_n, ctl);  // both halves have read the stored LSE
+  __nv_bfloat16* out_row = nullptr;
+  if (EPI == kEpiOut || EPI == kEpiAccOut)
+    out_row = static_cast<__nv_bfloat16*>(w.o) + it.b * w.o_sb + it.h * w.o_sh + it.r * w.o_rs +
+              static_cast<long long>(t) * w.o_ts;
+  const float wp = w_part * inv_l;
+#pragma unroll
+  for (int cc = 0; cc < HD / CH; ++cc) {
+    const int col0 = half * HD + cc * CH;
+    uint32_t orow[CH];
+    if (has_o) {
+      if constexpr (CH == 32)
+        tmem_ld32(o_addr + col0, orow);
+      else
+        tmem_ld16(o_addr + col0, orow);
+      tmem_ld_wait(orow);
+    } else {
+#pragma unroll
+      for (int e = 0; e < CH; ++e) orow[e] = 0u;
+    }
+    if (row_ok && !skip) {
+      float vals[CH];
+#pragma unroll
+      for (int e = 0; e < CH; ++e) vals[e] = __uint_as_float(orow[e]) * wp;
+      if (EPI == kEpiAcc || EPI == kEpiAccOut) {
+#pragma unroll
+        for (int e = 0; e < CH; e += 4) {
+          if (col0 + e < w.d) {
+            const float4 a = *reinterpret_cast<const float4*>(acc_row + col0 + e);
+            vals[e] = fmaf(w_acc, a.x, vals[e]);
+            vals[e + 1] = fmaf(w_acc, a.y, vals[e + 1]);
+            vals[e + 2] = fmaf(w_acc, a.z, vals[e + 2]);
+            vals[e + 3] = fmaf(w_acc, a.w, vals[e + 3]);
+          }
+        }
+      }
+      if (EPI == kEpiPart || EPI == kEpiAcc) {
+#pragma unroll
+        for (int e = 0; e < CH; e += 4)
+          if (col0 + e < w.d)
+            *reinterpret_cast<float4*>(acc_row + col0 + e) = make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < CH; e += 8) {
+          if (col0 + e < w.d) {
+            uint4 pkt;
+            pkt.x = pack_bf16x2(vals[e], vals[e + 1]);
+            pkt.y = pack_bf16x2(vals[e + 2], vals[e + 3]);
+            pkt.z = pack_bf16x2(vals[e + 4], vals[e + 5]);
+            pkt.w = pack_bf16x2(vals[e + 6], vals[e + 7]);
+            *reinterpret_cast<uint4*>(out_row + col0 + e) = pkt;
+          }
+        }
+      }
+    }
+  }
+  if (row_ok && !skip && half == 0) {
+    if (EPI == kEpiPart || EPI == kEpiAcc) {
+      *accl_ptr = L;
+    } else if (w.lse != nullptr) {
+      w.lse[it.b * w.l_sb + it.h * w.l_sh + it.r * w.l_rs + static_cast<long long>(t) * w.l_ts] = L;
+    }
+  }
+}
+
 // p = 2^(s * scale_log2 - base) for the scores of column pairs [E0, E1) of this row, packed to
 // bf16 pairs in pk (the row of P_q); row sums accumulated in two packed fp32x2 chains.  EVERY > 0: one column pair in
 // EVERY goes to the FMA-pipe polynomial instead of the MUFU (only for tiles without masked
@@ -554,7 +697,7 @@ __device__ __forceinline__ void softmax_exp_store(const uint32_t (&sr)[NSC][32],
 // The kernel
 // ---------------------------------------------------------------------------------------------
 template <int DP, int EPI, bool WIN>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(FmhaCfg<DP>::THREADS, 1)
     fmha_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnWork w, int n_steps, int n_items) {
   using C = FmhaCfg<DP>;
@@ -582,10 +725,14 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_plan_full = bar_s_free + 2;         // [2] item plan slot written
   uint64_t* bar_plan_empty = bar_plan_full + 2;     // [2] item plan slot read by every consumer
   uint64_t* bar_exp_done = bar_plan_empty + 2;      // [2] softmax warpgroup q finished an exponential phase
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_exp_done + 2);
+  uint64_t* bar_pair = bar_exp_done + 2;            // [2] column-split halves of tile q meet (256 threads)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_pair + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* stats = reinterpret_cast<float2*>(tmem_slot + 4);  // [2][128] (m_used, l_sum)
   ItemPlan* plan = reinterpret_cast<ItemPlan*>(stats + 2 * 128);  // [2], slot = item sequence & 1
+  // Column-split softmax: row maxima [2 tile parity][2 q][2 half][128] and row sums [2 item
+  // parity][2 q][2 half][128] of the two halves of each row.
+  float* xch = reinterpret_cast<float*>(plan + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -602,21 +749,23 @@ __global__ void __launch_bounds__(512, 1)
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar_s_full + q, 1);
-      mbar_init(bar_p_full + q, 128);
+      constexpr int kHalves = C::SPLIT ? 2 : 1;
+      mbar_init(bar_p_full + q, C::SPLIT && kSplitWarpArrive ? 8 : 128 * kHalves);
       mbar_init(bar_pv_done + q, 1);
       mbar_init(bar_o_full + q, 1);
-      mbar_init(bar_o_empty + q, 128);
+      mbar_init(bar_o_empty + q, 128 * kHalves);
       mbar_init(bar_stats + q, 128);
-      mbar_init(bar_s_free + q, 128);
-      // Readers of a plan slot (d <= 64): each MMA issuer thread, 8 softmax warps, 4 epilogue warps.
+      mbar_init(bar_s_free + q, C::SPLIT && kSplitWarpArrive ? 8 : 128 * kHalves);
+      // Readers of a plan slot: each MMA issuer thread, every softmax warp, the 4 epilogue warps.
       mbar_init(bar_plan_full + q, 1);
-      mbar_init(bar_plan_empty + q, C::ISSUERS + 12);
+      mbar_init(bar_plan_empty + q, C::ISSUERS + C::SM_WARPS + (C::SPLIT ? 0 : 4));
       mbar_init(bar_exp_done + q, 4);  // one arrival per softmax warp
+      mbar_init(bar_pair + q, 8);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 12 && lane == 0) {
+  if (warp == C::PROD_WARP && lane == 0) {
     tma_prefetch_map(&tm_q);
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
@@ -630,9 +779,9 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 12) {
+  if (warp >= C::PROD_WARP) {
     setmaxnreg_dec<RegSplit<DP, EPI>::kProd>();
-    if (warp == 12 && lane == 0) {
+    if (warp == C::PROD_WARP && lane == 0) {
       // ================================================================ TMA producer
       int it_q = 0, it_seq = 0;
       long long g = 0;
@@ -690,7 +839,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_drain(bar_k_full + j % C::STAGES, static_cast<uint32_t>(j / C::STAGES) & 1, w.wait_limit_ns);
         mbar_drain(bar_v_full + j % C::STAGES, static_cast<uint32_t>(j / C::STAGES) & 1, w.wait_limit_ns);
       }
-    } else if (!C::P_SEP && warp == 13 && lane == 0) {
+    } else if (!C::P_SEP && warp == C::PROD_WARP + 1 && lane == 0) {
       // ================================================================ MMA issuer (P over S)
       // One thread, fixed order per key tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).  QK_q(j+1)
       // rewrites S_q, which holds P_q(j), so it waits for PV_q(j) to complete; meanwhile the
@@ -770,7 +919,7 @@ __global__ void __launch_bounds__(512, 1)
       // Tensor memory is freed only after every MMA issued here has completed.
       mma_commit(bar_mma_done);
       mbar_drain(bar_mma_done, 0, w.wait_limit_ns);
-    } else if (C::P_SEP && (warp == 13 || warp == 14) && lane == 0) {
+    } else if (C::P_SEP && (warp == C::PROD_WARP + 1 || warp == C::PROD_WARP + 2) && lane == 0) {
       // ================================================================ MMA issuers
       // One thread per query tile q (warp 13: q = 0, warp 14: q = 1).  Each blocks on its own next
       // event and issues, per key tile j:
@@ -782,7 +931,7 @@ __global__ void __launch_bounds__(512, 1)
       // A K/V stage is released when both issuers have committed it (kv_empty counts 2), and Q
       // when both have issued their last QK of the item (q_empty counts 2).  The issuer that is
       // behind never waits on the one ahead, so the two cannot deadlock.
-      const int q = warp - 13;
+      const int q = warp - (C::PROD_WARP + 1);
       constexpr uint32_t idesc_qk = make_idesc_bf16(128, C::BN, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, DP, 0, 1);
       const uint32_t q_addr = smem_addr(sQ) + q * C::Q_TILE_BYTES;
@@ -848,7 +997,186 @@ __global__ void __launch_bounds__(512, 1)
       mma_commit(bar_mma_done);
       mbar_drain(bar_mma_done, 0, w.wait_limit_ns);
     }
+  } else if (C::SPLIT) {
+    if constexpr (C::SPLIT) {
+      setmaxnreg_inc<RegSplit<DP, EPI>::kSoftmax>();
+      // ============================================================ softmax, column-split
+      // Warps 0-3 / 4-7: query tile 0 / 1, S columns [0, BN/2); warps 8-11 / 12-15: the same tiles,
+      // columns [BN/2, BN).  Thread = row = tensor-memory lane, as in the unsplit softmax.
+      const int q = (warp >> 2) & 1;
+      const int half = warp >> 3;
+      const int row = threadIdx.x & 127;
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      const uint32_t s_addr = lane_addr + C::S_COL0 + C::S_STRIDE * q + half * C::HCOLS;
+      const uint32_t p_addr = lane_addr + C::P_COL0 + C::P_STRIDE * q + half * (C::HCOLS / 2);
+      const uint32_t o_addr = lane_addr + C::O_COL0 + C::O_STRIDE * q;
+      float* xmax = xch;                  // [2][2][2][128]
+      float* xsum = xch + 2 * 2 * 2 * 128;  // [2][2][2][128]
+      const float sl2 = w.scale_log2;
+      constexpr int NH = C::HCOLS / 32;   // 32-column chunks of this half of an S row
+      constexpr int HD = C::D / 2;        // O columns of this half
+      constexpr int OCH = HD < 32 ? HD : 32;
+      int it_all = 0, c = 0, meets = 0;
+      bool ok = true;
+      bool s_seen = false;  // S_q of tile c already seen complete
+      for (int k = 0; ok && k * static_cast<int>(gridDim.x) < n_items; ++k) {
+        const int idx = item_of_cta(k);
+        if (idx >= n_items) continue;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_plan_full + (it_all & 1), (it_all >> 1) & 1, ctl, 0x305));
+        if (!ok) break;
+        const Item it = plan[it_all & 1].it;
+        const bool has_o = plan[it_all & 1].n > 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_plan_empty + (it_all & 1));
+        const bool row_ok = row < it.rows_valid[q];
+        const long long pos_q = it.pos0 + static_cast<long long>(it.t0 + 128 * q + row) * w.q_tstride;
+        float m_used = -INFINITY;  // running max of scaled scores, log2 units (same in both halves)
+        float l_sum = 0.f;         // running sum of 2^(x - m_used) over this half's columns
+        Walk wk;
+        int cur_s = -1, row_lim = 0, row_lo = 0;
+        for (bool has = walk_begin<WIN, C::BN>(wk, w, it, n_steps); has; has = walk_next<WIN, C::BN>(wk, w, it, n_steps)) {
+          if (wk.s != cur_s) {
+            cur_s = wk.s;
+            row_lim = row_ok ? visible_key_limit(w, pos_q, wk.s) : w.n_kv;
+            if (WIN) row_lo = row_ok ? visible_key_start(w, pos_q, wk.s) : 0;
+          }
+          if (!__all_sync(0xffffffffu, s_seen)) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + q, c & 1, ctl, 0x301));
+            if (!ok) break;
+          }
+          s_seen = false;
+          tc_fence_after();
+          uint32_t sr[NH][32];
+#pragma unroll
+          for (int cc = 0; cc < NH; ++cc) tmem_ld32(s_addr + cc * 32, sr[cc]);
+          tmem_ld_wait(sr[0]);
+#pragma unroll
+          for (int cc = 1; cc < NH; ++cc) reg_dep(sr[cc]);
+          tc_fence_before();
+          if (kSplitWarpArrive) {  // the next QK_q may overwrite S_q once both halves hold it
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_s_free + q);
+          } else {
+            mbar_arrive(bar_s_free + q);
+          }
+          const int c0 = wk.u0 + half * C::HCOLS;  // key of this half's first column
+          const int lim = row_lim - c0;            // columns [lo, lim) of this half are visible
+          const int lo = WIN ? row_lo - c0 : 0;
+          const bool cut = WIN ? (lim < C::HCOLS || lo > 0) : lim < C::HCOLS;
+          const bool masked = __any_sync(0xffffffffu, cut);
+          if (cut) {
+#pragma unroll
+            for (int e = 0; e < C::HCOLS; ++e)
+              if (e >= lim || (WIN && e < lo)) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
+          }
+          float mxp[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mxp[i] = __uint_as_float(sr[0][i]);
+#pragma unroll
+          for (int e = 8; e < C::HCOLS; e += 2)
+            mxp[(e >> 1) & 7] = fmax3(mxp[(e >> 1) & 7], __uint_as_float(sr[e >> 5][e & 31]),
+                                      __uint_as_float(sr[(e + 1) >> 5][(e + 1) & 31]));
+          const float mx_half =
+              fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
+          // Row max over both halves: exchange through shared memory (slot by tile parity).
+          float* xm = xmax + ((c & 1) * 4 + q * 2) * 128;
+          xm[half * 128 + row] = mx_half;
+          ok = __all_sync(0xffffffffu, pair_meet(bar_pair + q, meets, ctl));
+          if (!ok) break;
+          const float mx = fmaxf(mx_half, xm[(half ^ 1) * 128 + row]);
+          const float m_tile = mx * sl2;
+          float m_new = m_used;
+          float alpha = 1.f;
+          bool rescale = false;
+          if (m_tile > m_used) {
+            if (m_used == -INFINITY) {
+              m_new = m_tile;  // nothing accumulated yet in this item: this row of O is zero
+            } else if (m_tile > m_used + 8.f) {
+              m_new = m_tile;
+              alpha = ex2_approx(m_used - m_new);
+              rescale = true;
+            }
+          }
+          const float base = (m_new == -INFINITY) ? 0.f : m_new;
+          const bool any_rescale = __any_sync(0xffffffffu, rescale);
+          float2 rsp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // packed row sums
+          constexpr int HALF = NH * 8;  // column pairs in half of this half-row
+          uint32_t pk[NH * 16];
+          bool pv_seen;
+          if (masked || kEmuEvery == 0) {
+            softmax_exp<0, 0, HALF>(sr, sl2, base, pk, rsp);
+            pv_seen = c == 0 || mbar_test_wait(bar_pv_done + q, (c - 1) & 1);
+            softmax_exp<0, HALF, 2 * HALF>(sr, sl2, base, pk, rsp);
+          } else {
+            softmax_exp<kEmuEvery, 0, HALF>(sr, sl2, base, pk, rsp);
+            pv_seen = c == 0 || mbar_test_wait(bar_pv_done + q, (c - 1) & 1);
+            softmax_exp<kEmuEvery, HALF, 2 * HALF>(sr, sl2, base, pk, rsp);
+          }
+          s_seen = mbar_test_wait(bar_s_full + q, (c + 1) & 1);  // the next QK_q, issued at s_free
+          if (!__all_sync(0xffffffffu, pv_seen)) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + q, (c - 1) & 1, ctl, 0x302));
+            if (!ok) break;
+          }
+          tc_fence_after();
+          if constexpr (NH == 2)
+            tmem_st32(p_addr, pk);
+          else
+            tmem_st16(p_addr, pk);
+          if (any_rescale) {
+            // This half's columns of O (the previous PV_q has landed: its wait is above).
+#pragma unroll
+            for (int cc = 0; cc < HD / OCH; ++cc) {
+              const uint32_t a = o_addr + half * HD + cc * OCH;
+              uint32_t orow[OCH];
+              if constexpr (OCH == 32)
+                tmem_ld32(a, orow);
+              else
+                tmem_ld16(a, orow);
+              tmem_ld_wait(orow);
+#pragma unroll
+              for (int e = 0; e < OCH; e += 2) {
+                const float2 v = __fmul2_rn(make_float2(__uint_as_float(orow[e]), __uint_as_float(orow[e + 1])),
+                                            make_float2(alpha, alpha));
+                orow[e] = __float_as_uint(v.x);
+                orow[e + 1] = __float_as_uint(v.y);
+              }
+              if constexpr (OCH == 32)
+                tmem_st32(a, orow);
+              else
+                tmem_st16(a, orow);
+            }
+          }
+          l_sum = l_sum * alpha + ((rsp[0].x + rsp[0].y) + (rsp[1].x + rsp[1].y));
+          m_used = m_new;
+          tmem_st_wait();
+          tc_fence_before();
+          if (kSplitWarpArrive) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_p_full + q);
+          } else {
+            mbar_arrive(bar_p_full + q);
+          }
+          ++c;
+        }
+        if (!ok) break;
+        // Epilogue of this item's tile q: the row sum over both halves, then O / l and the LSE.
+        float* xs = xsum + ((it_all & 1) * 4 + q * 2) * 128;
+        xs[half * 128 + row] = l_sum;
+        ok = __all_sync(0xffffffffu, pair_meet(bar_pair + q, meets, ctl));
+        if (!ok) break;
+        const float l_row = l_sum + xs[(half ^ 1) * 128 + row];
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_full + q, it_all & 1, ctl, 0x401));
+        if (!ok) break;
+        tc_fence_after();
+        fmha_epilogue_row_half<C, EPI>(w, it, it.t0 + 128 * q + row, row_ok, has_o, make_float2(m_used, l_row),
+                                       o_addr, half, bar_pair + q, meets, ctl);
+        tc_fence_before();
+        mbar_arrive(bar_o_empty + q);
+        ++it_all;
+      }
+    }
   } else if (warp < 8) {
+   if constexpr (!C::SPLIT) {
     setmaxnreg_inc<RegSplit<DP, EPI>::kSoftmax>();
     // ================================================================ softmax (query tile q)
     const int q = warp >> 2;
@@ -1027,7 +1355,9 @@ __global__ void __launch_bounds__(512, 1)
       mbar_arrive(bar_stats + q);
       ++it_all;
     }
+   }
   } else {
+   if constexpr (!C::SPLIT) {
     setmaxnreg_dec<RegSplit<DP, EPI>::kEpi>();
     // ================================================================ epilogue (both tiles)
     const int row = threadIdx.x & 127;
@@ -1065,6 +1395,7 @@ __global__ void __launch_bounds__(512, 1)
       }
       ++it_all;
     }
+   }
   }
 
   tc_fence_before();
