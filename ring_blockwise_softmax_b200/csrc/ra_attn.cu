@@ -264,7 +264,10 @@ int heads_per_group(const ra::AttnWork& w, int elem_bytes) {
   const long long bh = static_cast<long long>(w.B) * w.H;
   const double whole = 80.0 * 1024 * 1024;
   if (kv_bytes * static_cast<double>(bh) <= whole) return static_cast<int>(bh);
-  const double budget = 40.0 * 1024 * 1024;
+#ifndef RA_L2_GROUP_MIB
+#define RA_L2_GROUP_MIB 40
+#endif
+  const double budget = static_cast<double>(RA_L2_GROUP_MIB) * 1024 * 1024;
   long long hg_max = static_cast<long long>(budget / (kv_bytes > 1.0 ? kv_bytes : 1.0));
   if (hg_max < 1) hg_max = 1;
   if (hg_max >= bh) return static_cast<int>(bh);
@@ -933,6 +936,15 @@ ra_status_t ra_attn_bwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_ten
     tw.wait_limit_ns = g_wait_limit_ns.load();
     tw.dev_status = dev.status;
     ra::BwdTcWork wq = tw, wkv = tw;
+    // One heavy-first order over all heads for causal launches of at most 32 waves of CTAs (load
+    // balance matters there; longer launches balance anyway and keep each head's CTAs together).
+    {
+      const long long waves = 32LL * (dev.sms > 0 ? dev.sms : 148);
+      const long long cq = static_cast<long long>((w.n_q + 127) / 128) * w.H * w.B;
+      const long long ckv = static_cast<long long>((w.n_kv + 127) / 128) * w.H_kv * w.B;
+      wq.global_order = w.causal && cq <= waves;
+      wkv.global_order = w.causal && ckv <= waves;
+    }
     wq.out1 = w.dq;
     wq.o1_sb = w.dq_sb;
     wq.o1_sh = w.dq_sh;

@@ -59,6 +59,7 @@ struct BwdTcWork {
   long long o2_sb, o2_sh, o2_st;
   unsigned long long wait_limit_ns;
   unsigned int* dev_status;
+  int global_order;  // remap CTAs to one heavy-first order over all heads (see bwd_range)
 };
 
 template <int DP, bool KV>
@@ -117,12 +118,29 @@ struct BwdRange {
 template <bool KV>
 __device__ __forceinline__ BwdRange bwd_range(const BwdTcWork& w) {
   BwdRange r;
-  r.b = blockIdx.z;
-  r.hf = blockIdx.y;
+  // CTAs start in linear block order (x fastest), heavy-first within each head.  With
+  // w.global_order the linear index is remapped so that the heaviest blocks of every head come
+  // first, then the next heaviest of every head, and so on: one global heavy-first order, which
+  // balances causal work over the SMs better (B=2 H=16 N=8192 d=64: +4 %) but spreads the CTAs
+  // running at one time over every head, which costs L2 locality (B=1 H=32 N=32768 d=128: -4 %).
+  // The host sets it for causal launches of few waves of CTAs, where the balance matters.
+  int level;  // 0 = heaviest
+  if (w.global_order) {
+    const int lin = static_cast<int>(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    const int nhb = static_cast<int>(gridDim.y * gridDim.z);
+    level = lin / nhb;
+    const int hb = lin - level * nhb;
+    r.b = hb / static_cast<int>(gridDim.y);
+    r.hf = hb - r.b * static_cast<int>(gridDim.y);
+  } else {
+    level = static_cast<int>(blockIdx.x);
+    r.b = static_cast<int>(blockIdx.z);
+    r.hf = static_cast<int>(blockIdx.y);
+  }
   constexpr int BM = 128, BN = 64;
   if (KV) {
-    // Key blocks in launch order: the first ones are seen by the most query rows (causal).
-    r.m0 = blockIdx.x * BM;
+    // Key blocks: the first ones are seen by the most query rows (causal).
+    r.m0 = level * BM;
     const int m_last = min(r.m0 + BM, w.n_kv) - 1;
     const int lo = w.causal ? r.m0 : 0;
     int hi = w.n_q;
@@ -132,7 +150,7 @@ __device__ __forceinline__ BwdRange bwd_range(const BwdTcWork& w) {
     r.te = lo < hi ? (hi + BN - 1) / BN : r.tb;
   } else {
     // Query blocks last-first: under a causal mask the last rows see the most keys.
-    r.m0 = (gridDim.x - 1 - blockIdx.x) * BM;
+    r.m0 = (static_cast<int>(gridDim.x) - 1 - level) * BM;
     const int m_last = min(r.m0 + BM, w.n_q) - 1;
     const int hi = w.causal ? min(w.n_kv, m_last + 1) : w.n_kv;
     int lo = 0;
