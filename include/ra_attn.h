@@ -213,6 +213,31 @@ ra_status_t ra_ring_fwd_window(const ra_tensor_t* q, const ra_tensor_t* k, const
                                const ra_tensor_t* o, float* lse, const ra_stream_t* streams,
                                int n_streams, void* workspace, size_t workspace_bytes);
 
+/* ra_ring_fwd for inputs and outputs that live in host memory, with the transfers overlapped with
+ * the computation.  There is no counterpart on the source pages: this is an interface convenience
+ * of this library, for callers whose tensors are host-resident (and, on the pages' multi-device
+ * ring, for a rank that receives its shards from the host).
+ * The flattened B*H_kv heads are split into n_chunks chunks (fewer when there are fewer heads);
+ * chunk c's query, key and value heads go host -> device on streams[0], its ring runs (fused
+ * schedule) on streams[1] as soon as they have landed, and its O and LSE go device -> host on
+ * streams[2] as soon as it is done, so chunk c+1's copies in and chunk c-1's copies out overlap
+ * chunk c's kernels.  Attention is independent per head, so the result equals ra_ring_fwd on the
+ * whole tensors.
+ * q_host, k_host, v_host, o_host: contiguous [B,H,N,d] (k, v: [B,H_kv,N,d]) tensors in host memory;
+ * page-locked memory is needed for the copies to overlap (pageable memory gives the same result,
+ * without the overlap).  q_dev .. o_dev: device tensors of the same shapes and dtypes, contiguous
+ * (caller-allocated staging; every chunk has its own region, nothing is reused within the call).
+ * lse_host, lse_dev: fp32 [B,H,N], both given or both NULL.  streams: three distinct caller-owned
+ * streams (copy in, compute, copy out).  The call orders itself after work already queued on
+ * streams[1]; on return every part of it, the copies out included, is ordered before later work
+ * on streams[1], so synchronising streams[1] makes o_host and lse_host valid.  Every check runs
+ * before anything is enqueued; RA_ERR_CUDA from a failed copy or launch in the middle leaves the
+ * earlier chunks queued.  Other arguments and errors as for ra_ring_fwd. */
+ra_status_t ra_ring_fwd_host(const ra_tensor_t* q_host, const ra_tensor_t* k_host, const ra_tensor_t* v_host, int P,
+                             int layout, int causal, float scale, const ra_tensor_t* o_host, float* lse_host,
+                             const ra_tensor_t* q_dev, const ra_tensor_t* k_dev, const ra_tensor_t* v_dev,
+                             const ra_tensor_t* o_dev, float* lse_dev, int n_chunks, const ra_stream_t* streams);
+
 /* ra_ring_fwd with the RA_RING_STEPWISE schedule for callers that cannot allocate device memory
  * at the point of the call: code inside a host application whose caching allocator already holds
  * all device memory and offers no scratch interface, services that fix their memory budget at

@@ -663,10 +663,11 @@ ra_status_t ra_ring_workspace_size(const ra_tensor_t* q, int P, int schedule, si
   return ok();
 }
 
+// dry_run: every check of the call, encoding and launch preparation included, and nothing enqueued.
 static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, int P,
                                  int layout, int causal, int64_t window, float scale, int schedule,
                                  const ra_tensor_t* o, float* lse, const ra_stream_t* streams, int n_streams,
-                                 void* workspace, size_t workspace_bytes) {
+                                 void* workspace, size_t workspace_bytes, bool dry_run = false) {
   ra_status_t st = check_qkv(q, k, v);
   if (st != RA_OK) return st;
   if ((st = check_out(o, q, "o", q->dtype)) != RA_OK) return st;
@@ -763,6 +764,7 @@ static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, con
   }
   for (Launch& l : launches)
     if ((st = prepare_attention(q, l.w, l.n_steps, &l.w)) != RA_OK) return st;
+  if (dry_run) return ok();
 
   // Events that fork the extra streams off streams[0] (so the call is ordered after work already
   // queued there) and join them back, created before anything is enqueued.
@@ -840,6 +842,137 @@ ra_status_t ra_ring_fwd_window(const ra_tensor_t* q, const ra_tensor_t* k, const
   if (window < 1) return fail(RA_ERR_INVALID_ARG, "window must be >= 1 (got %lld)", (long long)window);
   return ring_fwd_impl(q, k, v, P, layout, 1, window, scale, schedule, o, lse, streams, n_streams, workspace,
                        workspace_bytes);
+}
+
+// A contiguous [B, H, N, d] tensor: stride = (H*N*d, N*d, d, 1).
+static bool packed_4d(const ra_tensor_t* t) {
+  return t->stride[3] == 1 && t->stride[2] == t->shape[3] && t->stride[1] == t->shape[2] * t->shape[3] &&
+         (t->shape[0] == 1 || t->stride[0] == t->shape[1] * t->shape[2] * t->shape[3]);
+}
+
+// Heads [h0, h0 + nh) of the flattened B*H heads of a contiguous tensor, as a [1, nh, N, d] view.
+static ra_tensor_t head_chunk(const ra_tensor_t* t, int64_t h0, int64_t nh) {
+  ra_tensor_t c = *t;
+  const int64_t per_head = t->shape[2] * t->shape[3];
+  const size_t elem = t->dtype == RA_BF16 ? 2 : 4;
+  c.data = static_cast<char*>(t->data) + static_cast<size_t>(h0 * per_head) * elem;
+  c.shape[0] = 1;
+  c.shape[1] = nh;
+  c.stride[0] = nh * per_head;
+  c.stride[1] = per_head;
+  return c;
+}
+
+ra_status_t ra_ring_fwd_host(const ra_tensor_t* q_host, const ra_tensor_t* k_host, const ra_tensor_t* v_host, int P,
+                             int layout, int causal, float scale, const ra_tensor_t* o_host, float* lse_host,
+                             const ra_tensor_t* q_dev, const ra_tensor_t* k_dev, const ra_tensor_t* v_dev,
+                             const ra_tensor_t* o_dev, float* lse_dev, int n_chunks, const ra_stream_t* streams) {
+  const ra_tensor_t* hosts[4] = {q_host, k_host, v_host, o_host};
+  const ra_tensor_t* devs[4] = {q_dev, k_dev, v_dev, o_dev};
+  const char* names[4] = {"q", "k", "v", "o"};
+  ra_status_t st;
+  for (int i = 0; i < 4; ++i) {
+    if ((st = check_tensor(hosts[i], names[i])) != RA_OK) return st;
+    if ((st = check_tensor(devs[i], names[i])) != RA_OK) return st;
+    if (!packed_4d(hosts[i]) || !packed_4d(devs[i]))
+      return fail(RA_ERR_UNSUPPORTED, "%s: host and device tensors must be contiguous [B, H, N, d]", names[i]);
+    if (hosts[i]->dtype != devs[i]->dtype)
+      return fail(RA_ERR_INVALID_ARG, "%s: host and device tensors differ in dtype", names[i]);
+    for (int a = 0; a < 4; ++a)
+      if (hosts[i]->shape[a] != devs[i]->shape[a])
+        return fail(RA_ERR_INVALID_ARG, "%s: host and device tensors differ in shape", names[i]);
+  }
+  if ((lse_host == nullptr) != (lse_dev == nullptr))
+    return fail(RA_ERR_INVALID_ARG, "lse_host and lse_dev must both be given or both be NULL");
+  if (streams == nullptr || streams[0] == streams[1] || streams[1] == streams[2] || streams[0] == streams[2])
+    return fail(RA_ERR_INVALID_ARG, "three distinct streams are needed (copy in, compute, copy out)");
+  if (n_chunks < 1) return fail(RA_ERR_INVALID_ARG, "n_chunks must be >= 1");
+  const int64_t kv_heads = k_dev->shape[0] * k_dev->shape[1];  // flattened K/V heads
+  if (k_dev->shape[1] < 1 || q_dev->shape[1] % k_dev->shape[1] != 0)
+    return fail(RA_ERR_INVALID_ARG, "H_kv must divide H");
+  const int64_t qpk = q_dev->shape[1] / k_dev->shape[1];
+  const int64_t chunks = n_chunks < kv_heads ? n_chunks : kv_heads;
+  // Chunk c: K/V heads [c*G/n, (c+1)*G/n) of the flattened B*H_kv, and their qpk query heads each.
+  auto bounds = [&](int64_t c, int64_t* k0, int64_t* nk) {
+    *k0 = c * kv_heads / chunks;
+    *nk = (c + 1) * kv_heads / chunks - *k0;
+  };
+  // Every check of the per-chunk ring call before anything is enqueued (chunks differ only in
+  // their head count, so the first and the largest one cover them all).
+  const ra_stream_t compute[1] = {streams[1]};
+  for (int64_t c : {int64_t(0), chunks - 1}) {
+    int64_t k0, nk;
+    bounds(c, &k0, &nk);
+    ra_tensor_t qc = head_chunk(q_dev, k0 * qpk, nk * qpk), kc = head_chunk(k_dev, k0, nk),
+                vc = head_chunk(v_dev, k0, nk), oc = head_chunk(o_dev, k0 * qpk, nk * qpk);
+    if ((st = ring_fwd_impl(&qc, &kc, &vc, P, layout, causal, 0, scale, RA_RING_FUSED, &oc,
+                            lse_dev ? lse_dev + k0 * qpk * q_dev->shape[2] : nullptr, compute, 1, nullptr, 0,
+                            true)) != RA_OK)
+      return st;
+  }
+  const cudaStream_t s_in = reinterpret_cast<cudaStream_t>(streams[0]);
+  const cudaStream_t s_cmp = reinterpret_cast<cudaStream_t>(streams[1]);
+  const cudaStream_t s_out = reinterpret_cast<cudaStream_t>(streams[2]);
+  std::vector<cudaEvent_t> ev(2 * chunks + 2, nullptr);
+  cudaError_t e = cudaSuccess;
+  for (auto& x : ev)
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+  auto destroy = [&ev] {
+    for (cudaEvent_t x : ev)
+      if (x) cudaEventDestroy(x);
+  };
+  if (e != cudaSuccess) {
+    destroy();
+    return cuda_fail(e, "event");
+  }
+  // The copies wait for work already queued on the compute stream (which may still use the
+  // device buffers).
+  e = cudaEventRecord(ev[2 * chunks], s_cmp);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev[2 * chunks], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev[2 * chunks], 0);
+  if (e != cudaSuccess) {
+    destroy();
+    return cuda_fail(e, "stream fork");
+  }
+  const size_t lse_row = static_cast<size_t>(q_dev->shape[2]) * sizeof(float);
+  for (int64_t c = 0; c < chunks && st == RA_OK; ++c) {
+    int64_t k0, nk;
+    bounds(c, &k0, &nk);
+    const ra_tensor_t qh = head_chunk(q_host, k0 * qpk, nk * qpk), kh = head_chunk(k_host, k0, nk),
+                      vh = head_chunk(v_host, k0, nk), oh = head_chunk(o_host, k0 * qpk, nk * qpk);
+    ra_tensor_t qc = head_chunk(q_dev, k0 * qpk, nk * qpk), kc = head_chunk(k_dev, k0, nk),
+                vc = head_chunk(v_dev, k0, nk), oc = head_chunk(o_dev, k0 * qpk, nk * qpk);
+    const size_t elem = q_dev->dtype == RA_BF16 ? 2 : 4;
+    const size_t qbytes = static_cast<size_t>(nk * qpk * q_dev->shape[2] * q_dev->shape[3]) * elem;
+    const size_t kbytes = static_cast<size_t>(nk * k_dev->shape[2] * k_dev->shape[3]) * elem;
+    e = cudaMemcpyAsync(qc.data, qh.data, qbytes, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(kc.data, kh.data, kbytes, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(vc.data, vh.data, kbytes, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[2 * c], s_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_cmp, ev[2 * c], 0);
+    if (e != cudaSuccess) {
+      st = cuda_fail(e, "host-to-device copy");
+      break;
+    }
+    float* lc = lse_dev ? lse_dev + k0 * qpk * q_dev->shape[2] : nullptr;
+    if ((st = ring_fwd_impl(&qc, &kc, &vc, P, layout, causal, 0, scale, RA_RING_FUSED, &oc, lc, compute, 1, nullptr,
+                            0)) != RA_OK)
+      break;
+    e = cudaEventRecord(ev[2 * c + 1], s_cmp);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev[2 * c + 1], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(oh.data, oc.data, qbytes, cudaMemcpyDeviceToHost, s_out);
+    if (e == cudaSuccess && lse_host)
+      e = cudaMemcpyAsync(lse_host + k0 * qpk * q_dev->shape[2], lc, static_cast<size_t>(nk * qpk) * lse_row,
+                          cudaMemcpyDeviceToHost, s_out);
+    if (e != cudaSuccess) st = cuda_fail(e, "device-to-host copy");
+  }
+  // Later work on the compute stream is ordered after the whole call, the copies out included.
+  e = cudaEventRecord(ev[2 * chunks + 1], s_out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_cmp, ev[2 * chunks + 1], 0);
+  destroy();
+  if (st != RA_OK) return st;
+  if (e != cudaSuccess) return cuda_fail(e, "stream join");
+  return ok();
 }
 
 ra_status_t ra_attn_bwd(const ra_tensor_t* q, const ra_tensor_t* k, const ra_tensor_t* v, const ra_tensor_t* o,

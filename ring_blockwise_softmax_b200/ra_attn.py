@@ -42,7 +42,7 @@ SCHEDULES = {"stepwise": RA_RING_STEPWISE, "fused": RA_RING_FUSED}
 # Exported symbols of the library, in header order (the CPU test checks each one is present).
 SYMBOLS = (
     "ra_attn_fwd", "ra_attn_fwd_window", "ra_attn_bwd", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_workspace_size",
-    "ra_ring_fwd", "ra_ring_fwd_window", "ra_ring_fwd_noalloc", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
+    "ra_ring_fwd", "ra_ring_fwd_window", "ra_ring_fwd_host", "ra_ring_fwd_noalloc", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
     "ra_debug_exp2", "ra_status_string", "ra_last_error", "ra_version",
 )
 
@@ -73,6 +73,8 @@ _lib.ra_ring_fwd.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_in
 _lib.ra_ring_fwd_window.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_int,
                                     _T, _F, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_void_p,
                                     ctypes.c_size_t]
+_lib.ra_ring_fwd_host.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, _T, _F, _T, _T,
+                                  _T, _T, _F, ctypes.c_int, ctypes.POINTER(ctypes.c_void_p)]
 _lib.ra_ring_fwd_noalloc.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, _T, _F,
                                      _S]
 _lib.ra_get_device_status.argtypes = [_S]
@@ -246,6 +248,23 @@ def ring_fwd(q, k, v, P: int, layout: str, causal: bool, o, lse=None, scale: flo
     _check(_lib.ra_ring_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), int(P), LAYOUTS[layout],
                             int(bool(causal)), float(scale), SCHEDULES[schedule], ctypes.byref(to), _ptr(lse), arr,
                             len(streams), ws_ptr, ws_bytes), "ra_ring_fwd")
+
+
+def ring_fwd_host(q_host, k_host, v_host, P: int, layout: str, causal: bool, o_host, lse_host, q_dev, k_dev, v_dev,
+                  o_dev, lse_dev, scale: float = 0.0, n_chunks: int = 8, streams=None):
+    """ra_ring_fwd_host: host-resident inputs and outputs (pinned for overlap), device staging
+    tensors of the same shapes, three streams (copy in, compute, copy out; default: new ones)."""
+    import torch
+
+    if streams is None:
+        streams = [torch.cuda.Stream(device=q_dev.device) for _ in range(3)]
+    arr = (ctypes.c_void_p * 3)(*[(s if isinstance(s, int) else s.cuda_stream) for s in streams])
+    ts = [tensor_desc(x) for x in (q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev)]
+    _check(_lib.ra_ring_fwd_host(ctypes.byref(ts[0]), ctypes.byref(ts[1]), ctypes.byref(ts[2]), int(P), LAYOUTS[layout],
+                                 int(bool(causal)), float(scale), ctypes.byref(ts[3]), _ptr(lse_host),
+                                 ctypes.byref(ts[4]), ctypes.byref(ts[5]), ctypes.byref(ts[6]), ctypes.byref(ts[7]),
+                                 _ptr(lse_dev), int(n_chunks), arr), "ra_ring_fwd_host")
+    return streams
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20

@@ -143,3 +143,33 @@ def test_backward_host_validation(ra):
     assert call(o=to32) == ra.RA_ERR_INVALID_ARG and b"q's dtype" in lib.ra_last_error()
     k3 = ra.tensor_desc(torch.zeros(1, 3, 32, 64, dtype=torch.bfloat16))
     assert call(kk=k3) == ra.RA_ERR_INVALID_ARG
+
+
+def test_host_pipeline_validation(ra):
+    """ra_ring_fwd_host rejects bad arguments before anything reaches a device."""
+    import torch
+
+    lib = ra.lib_handle()
+    q = torch.zeros(1, 4, 64, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+    t = {n: ra.tensor_desc(x) for n, x in (("q", q), ("k", k), ("v", k), ("o", q))}
+    strided = ra.tensor_desc(q.transpose(1, 2).contiguous().transpose(1, 2))  # [B,H,N,d] view, not packed
+    f32 = ra.tensor_desc(q.float())
+    small = ra.tensor_desc(q[:, :2])
+    streams = (ctypes.c_void_p * 3)(1, 2, 3)
+    same = (ctypes.c_void_p * 3)(1, 1, 3)
+    lse = ctypes.c_void_p(16)
+
+    def call(qh=None, qd=None, lse_h=lse, lse_d=lse, chunks=2, st=streams):
+        qh = qh or t["q"]
+        qd = qd or t["q"]
+        return lib.ra_ring_fwd_host(ctypes.byref(qh), ctypes.byref(t["k"]), ctypes.byref(t["v"]), 4, 0, 1,
+                                    ctypes.c_float(0), ctypes.byref(t["o"]), lse_h, ctypes.byref(qd),
+                                    ctypes.byref(t["k"]), ctypes.byref(t["v"]), ctypes.byref(t["o"]), lse_d, chunks, st)
+
+    assert call(qh=strided) == ra.RA_ERR_UNSUPPORTED and b"contiguous" in lib.ra_last_error()
+    assert call(qd=f32) == ra.RA_ERR_INVALID_ARG and b"dtype" in lib.ra_last_error()
+    assert call(qd=small) == ra.RA_ERR_INVALID_ARG and b"shape" in lib.ra_last_error()
+    assert call(lse_d=None) == ra.RA_ERR_INVALID_ARG and b"both" in lib.ra_last_error()
+    assert call(st=same) == ra.RA_ERR_INVALID_ARG and b"distinct streams" in lib.ra_last_error()
+    assert call(chunks=0) == ra.RA_ERR_INVALID_ARG and b"n_chunks" in lib.ra_last_error()
