@@ -35,6 +35,13 @@
  *    refusing a kernel launch in the middle of a multi-launch ring call (ra_ring_fwd and its
  *    variants): the launches before it stay queued, and streams[0] is still ordered after them.
  *  - Device pointers must belong to the current CUDA device.
+ *  - Stream order holds as usual: work enqueued after a call, with an ordinary launch or copy,
+ *    starts after all of the call's work.  Inside a call, later steps of the stepwise ring and the
+ *    dK/dV half of the backward are launched as programmatic dependents of the kernel before them
+ *    (they start on SMs that kernel leaves idle and wait for it before touching its outputs); the
+ *    library's kernels signal dependents at their start, so a kernel of the caller's that is itself
+ *    launched as a programmatic dependent of a library call must wait for its grid dependency
+ *    before reading the call's outputs, as with any such launch.
  *
  * Supported inputs
  *  - dtype RA_BF16 (tensor-core path, fp32 accumulation, bf16 output): head dim d a multiple of 8

@@ -309,16 +309,16 @@ ra_status_t prepare_attention(const ra_tensor_t* q, const ra::AttnWork& w_in, in
 
 // Launches a work description completed by prepare_attention.
 ra_status_t launch_prepared(const ra_tensor_t* q, const Maps* maps, const ra::AttnWork& w, int n_steps, int epi,
-                            int sms, cudaStream_t stream) {
+                            int sms, cudaStream_t stream, bool dependent = false) {
   cudaError_t e;
   if (q->dtype == RA_BF16) {
     const int dp = padded_dim(w.d);
     if (dp == 32)
-      e = ra::launch_fmha_dp32(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream);
+      e = ra::launch_fmha_dp32(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream, dependent);
     else if (dp == 64)
-      e = ra::launch_fmha_dp64(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream);
+      e = ra::launch_fmha_dp64(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream, dependent);
     else
-      e = ra::launch_fmha_dp128(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream);
+      e = ra::launch_fmha_dp128(maps->q, maps->k, maps->v, w, n_steps, epi, sms, stream, dependent);
   } else {
     const long long gx = static_cast<long long>(w.n_q_tiles) * w.n_r;
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(w.H), static_cast<unsigned>(w.B));
@@ -745,6 +745,7 @@ static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, con
   struct Launch {
     ra::AttnWork w;
     int stream, n_steps, epi;
+    bool dependent;  // a later step of the stepwise ring on the same stream (tensor-core path)
   };
   std::vector<Launch> launches;
   for (int i = 0; i < n_streams; ++i) {
@@ -754,11 +755,15 @@ static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, con
     wi.n_r = (P - i + n_streams - 1) / n_streams;
     if (schedule == RA_RING_FUSED || P == 1) {
       wi.ring_step = 0;
-      launches.push_back({wi, i, P, ra::kEpiOut});
+      launches.push_back({wi, i, P, ra::kEpiOut, false});
     } else {
       for (int t = 0; t < P; ++t) {
         wi.ring_step = t;
-        launches.push_back({wi, i, 1, t == 0 ? ra::kEpiPart : (t == P - 1 ? ra::kEpiAccOut : ra::kEpiAcc)});
+#ifndef RA_PDL
+#define RA_PDL 1
+#endif
+        launches.push_back({wi, i, 1, t == 0 ? ra::kEpiPart : (t == P - 1 ? ra::kEpiAccOut : ra::kEpiAcc),
+                            RA_PDL && t > 0 && q->dtype == RA_BF16});
       }
     }
   }
@@ -797,7 +802,8 @@ static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, con
   st = RA_OK;
   std::string launch_error;
   for (const Launch& l : launches) {
-    st = launch_prepared(q, &maps, l.w, l.n_steps, l.epi, dev.sms, reinterpret_cast<cudaStream_t>(streams[l.stream]));
+    st = launch_prepared(q, &maps, l.w, l.n_steps, l.epi, dev.sms, reinterpret_cast<cudaStream_t>(streams[l.stream]),
+                         l.dependent);
     if (st != RA_OK) {
       launch_error = t_last_error;
       break;

@@ -10,6 +10,11 @@
 
 namespace ra {
 
+#ifndef RA_PDL
+#define RA_PDL 1
+#endif
+
+// kv (the dK/dV instance, launched after the dQ one): as a programmatic dependent of the dQ launch.
 template <class C, class K>
 static cudaError_t launch_kernel(K kern, bool kv, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b1,
                                  const CUtensorMap& b2, const CUtensorMap& b3, const BwdTcWork& w,
@@ -18,8 +23,21 @@ static cudaError_t launch_kernel(K kern, bool kv, const CUtensorMap& a1, const C
   if (e != cudaSuccess) return e;
   const int rows = kv ? w.n_kv : w.n_q;
   const dim3 grid((rows + C::BM - 1) / C::BM, kv ? w.H_kv : w.H, w.B);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(a1, a2, b1, b2, b3, w);
-  return cudaGetLastError();
+  if (!(kv && RA_PDL)) {
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(a1, a2, b1, b2, b3, w);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a1, a2, b1, b2, b3, w);
 }
 
 // The warpgroup ping-pong kernel wherever each warpgroup's (S, dP) buffer and P, dS columns fit

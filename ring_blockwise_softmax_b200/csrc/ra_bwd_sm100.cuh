@@ -267,6 +267,11 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The dK/dV launch follows the dQ launch as a programmatic dependent (the two read the same
+  // inputs and write different outputs), so its CTAs may fill SMs the dQ grid leaves idle at its
+  // end.  Every CTA waits for any such prerequisite grid before it exits (below), so neither
+  // launch completes before the one ahead of it on the stream.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 8) {
     if (lane == 0 && rg.n > 0) {
@@ -583,6 +588,7 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -698,6 +704,11 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The dK/dV launch follows the dQ launch as a programmatic dependent (the two read the same
+  // inputs and write different outputs), so its CTAs may fill SMs the dQ grid leaves idle at its
+  // end.  Every CTA waits for any such prerequisite grid before it exits (below), so neither
+  // launch completes before the one ahead of it on the stream.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 8) {
     if (lane == 0 && rg.n > 0) {
@@ -1009,6 +1020,7 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace ra

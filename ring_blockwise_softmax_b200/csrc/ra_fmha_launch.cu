@@ -11,7 +11,7 @@ namespace ra {
 
 template <int EPI, bool WIN>
 static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
-                              int n_steps, int sms, cudaStream_t stream) {
+                              int n_steps, int sms, cudaStream_t stream, bool dependent) {
   using C = FmhaCfg<RA_FMHA_DP>;
   auto kern = fmha_fwd_sm100<RA_FMHA_DP, EPI, WIN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -27,8 +27,23 @@ static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, cons
   const long long n_items = static_cast<long long>((w.n_q + C::ROWS - 1) / C::ROWS) * w.n_r * w.H * w.B;
   if (n_items > 2147483647LL) return cudaErrorInvalidValue;
   const int grid = static_cast<int>(n_items < sms ? n_items : sms);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, w, n_steps, static_cast<int>(n_items));
-  return cudaGetLastError();
+  if (!dependent) {
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, w, n_steps, static_cast<int>(n_items));
+    return cudaGetLastError();
+  }
+  // Programmatic dependent launch: this grid may start while the previous kernel on the stream
+  // (the previous ring step, which signals at its start) is finishing; its epilogue waits for it.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, w, n_steps, static_cast<int>(n_items));
 }
 
 #define RA_CAT2(a, b) a##b
@@ -36,22 +51,22 @@ static cudaError_t launch_epi(const CUtensorMap& mq, const CUtensorMap& mk, cons
 
 cudaError_t RA_CAT(launch_fmha_dp, RA_FMHA_DP)(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                                const AttnWork& w, int n_steps, int epi, int sms,
-                                               cudaStream_t stream) {
+                                               cudaStream_t stream, bool dependent) {
   // Launches with a sliding window use their own instantiation (WIN = true).
   const bool win = w.window > 0;
   switch (epi) {
     case kEpiOut:
-      return win ? launch_epi<kEpiOut, true>(mq, mk, mv, w, n_steps, sms, stream)
-                 : launch_epi<kEpiOut, false>(mq, mk, mv, w, n_steps, sms, stream);
+      return win ? launch_epi<kEpiOut, true>(mq, mk, mv, w, n_steps, sms, stream, dependent)
+                 : launch_epi<kEpiOut, false>(mq, mk, mv, w, n_steps, sms, stream, dependent);
     case kEpiPart:
-      return win ? launch_epi<kEpiPart, true>(mq, mk, mv, w, n_steps, sms, stream)
-                 : launch_epi<kEpiPart, false>(mq, mk, mv, w, n_steps, sms, stream);
+      return win ? launch_epi<kEpiPart, true>(mq, mk, mv, w, n_steps, sms, stream, dependent)
+                 : launch_epi<kEpiPart, false>(mq, mk, mv, w, n_steps, sms, stream, dependent);
     case kEpiAcc:
-      return win ? launch_epi<kEpiAcc, true>(mq, mk, mv, w, n_steps, sms, stream)
-                 : launch_epi<kEpiAcc, false>(mq, mk, mv, w, n_steps, sms, stream);
+      return win ? launch_epi<kEpiAcc, true>(mq, mk, mv, w, n_steps, sms, stream, dependent)
+                 : launch_epi<kEpiAcc, false>(mq, mk, mv, w, n_steps, sms, stream, dependent);
     case kEpiAccOut:
-      return win ? launch_epi<kEpiAccOut, true>(mq, mk, mv, w, n_steps, sms, stream)
-                 : launch_epi<kEpiAccOut, false>(mq, mk, mv, w, n_steps, sms, stream);
+      return win ? launch_epi<kEpiAccOut, true>(mq, mk, mv, w, n_steps, sms, stream, dependent)
+                 : launch_epi<kEpiAccOut, false>(mq, mk, mv, w, n_steps, sms, stream, dependent);
     default:
       return cudaErrorInvalidValue;
   }

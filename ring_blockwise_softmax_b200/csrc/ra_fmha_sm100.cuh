@@ -780,6 +780,10 @@ __global__ void __launch_bounds__(FmhaCfg<DP>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // A launch that follows this one on the stream with programmatic dependent launch (the next
+  // step of the stepwise ring) may be scheduled now: it takes SMs only as this grid's CTAs exit,
+  // and waits for this grid to finish before its epilogue touches memory this grid writes.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp >= C::PROD_WARP) {
     setmaxnreg_dec<RegSplit<DP, EPI>::kProd>();
@@ -1002,6 +1006,7 @@ __global__ void __launch_bounds__(FmhaCfg<DP>::THREADS, 1)
   } else if (C::SPLIT) {
     if constexpr (C::SPLIT) {
       setmaxnreg_inc<RegSplit<DP, EPI>::kSoftmax>();
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // runs the epilogue (see the epilogue role)
       // ============================================================ softmax, column-split
       // Warps 0-3 / 4-7: query tile 0 / 1, S columns [0, BN/2); warps 8-11 / 12-15: the same tiles,
       // columns [BN/2, BN).  Thread = row = tensor-memory lane, as in the unsplit softmax.
@@ -1362,6 +1367,9 @@ __global__ void __launch_bounds__(FmhaCfg<DP>::THREADS, 1)
    if constexpr (!C::SPLIT) {
     setmaxnreg_dec<RegSplit<DP, EPI>::kEpi>();
     // ================================================================ epilogue (both tiles)
+    // The only role that touches global memory other than Q, K, V: when launched as a dependent of
+    // the previous ring step, wait here for that grid to complete (returns at once otherwise).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = threadIdx.x & 127;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     int it_all = 0;

@@ -19,11 +19,11 @@ namespace ra {
 unsigned long long current_context_id();
 
 cudaError_t launch_fmha_dp32(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
-                             int n_steps, int epi, int sms, cudaStream_t stream);
+                             int n_steps, int epi, int sms, cudaStream_t stream, bool dependent);
 cudaError_t launch_fmha_dp64(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
-                             int n_steps, int epi, int sms, cudaStream_t stream);
+                             int n_steps, int epi, int sms, cudaStream_t stream, bool dependent);
 cudaError_t launch_fmha_dp128(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnWork& w,
-                              int n_steps, int epi, int sms, cudaStream_t stream);
+                              int n_steps, int epi, int sms, cudaStream_t stream, bool dependent);
 
 // Tensor maps of the tensor-core backward: 128-row boxes for the fixed operands of a CTA,
 // 64-row boxes for the streamed tiles.
