@@ -333,6 +333,8 @@ def config_dict(w, args):
 
     if w.N != I.WORKLOADS[w.cfg].N:
         name += f", sequence length reduced to {w.N}"
+    if w.layout != I.WORKLOADS[w.cfg].layout:
+        name += f", {w.layout} shards instead"
     return {"workload": f"cfg{w.cfg}: {name}", "B": w.B, "H": w.H, "H_kv": w.H_kv or w.H, "N": w.N, "d": w.d,
             "causal": w.causal, "window": w.window,
             "P": w.P, "layout": w.layout, "schedule": args.schedule,
@@ -646,6 +648,8 @@ def main(argv=None):
                     help="causal sliding-window variant of a causal workload (window in positions)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query variant of the workload: K and V with this many heads (must divide H)")
+    ap.add_argument("--layout", choices=["contiguous", "striped"], default=None,
+                    help="ring shard layout override (the workload's own by default)")
     ap.add_argument("--n", type=int, default=None,
                     help="sequence length override: a smaller case of the workload's layout (profiling)")
     ap.add_argument("--traffic", type=float, default=None,
@@ -656,6 +660,10 @@ def main(argv=None):
     from ring_blockwise_softmax_b200 import inputs as I
 
     w = I.WORKLOADS[args.config]
+    if args.layout is not None:
+        import dataclasses
+
+        w = dataclasses.replace(w, layout=args.layout)
     if args.n is not None:
         import dataclasses
 
