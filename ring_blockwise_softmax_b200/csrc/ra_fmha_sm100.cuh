@@ -2,13 +2,13 @@
 //
 // What it computes: the online softmax of intelliparadigm.com "深度学习注意力机制优化与
 // FlashAttention实践" §4.2 (with the output rescaled when the running max moves, which the
-// printed listing omits): K/V tiles of 128 keys stream through shared memory, S = Q K^T and
-// O += P V run as tcgen05 MMAs with fp32 accumulators in tensor memory, and a per-row running
-// max m and sum s are kept in fp32 registers.  One launch may walk several KV shards of a ring
-// in ring order (query shard r meets KV shard (r - t) mod P at step t, vibe-research.pages.dev
-// "Ring Attention" diagram); a shard boundary needs no extra work because the running
-// (m, s, O) already is the merged state of every shard seen so far (blog.gitcode.com
-// "分布式注意力机制突破…" §3.4: align the maxima, rescale the sums).
+// printed listing omits): K/V tiles stream through shared memory, S = Q K^T and O += P V run as
+// tcgen05 MMAs with fp32 accumulators in tensor memory, and a per-row running max m and sum s
+// are kept in fp32 registers.  One launch may walk several KV shards of a ring in ring order
+// (query shard r meets KV shard (r - t) mod P at step t, vibe-research.pages.dev "Ring
+// Attention" diagram); a shard boundary needs no extra work because the running (m, s, O)
+// already is the merged state of every shard seen so far (blog.gitcode.com "分布式注意力机制突破…"
+// §3.4: align the maxima, rescale the sums).
 //
 // Structure (persistent: one CTA per SM walks work items; an item is 256 query rows = two
 // 128-row query tiles of one (batch, head, query shard); items are numbered longest first and
@@ -16,25 +16,29 @@
 //   warps 0-3   softmax of query tile 0, thread i = row i = tensor-memory lane i
 //   warps 4-7   softmax of query tile 1
 //   warps 8-11  epilogue: normalise O, write O / LSE or LSE-merge into the accumulator
-//   warp 12     TMA producer: Q (two tiles) per item, then K_j / V_j into a STAGES-deep ring;
-//               for DP <= 64 it also publishes each item's decoded plan (ItemPlan) to the others
-//   warps 13,14 MMA issuers, one thread per query tile (DP <= 64): S_q = Q_q K_j^T (SS form),
-//               O_q += P_q V_j (TS form); for DP = 128 one thread in warp 13 issues both tiles'
-//               MMAs in the fixed order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1)
-// Both query tiles share every K/V tile (loaded once per 256 rows).  With P in its own columns
-// (DP <= 64) the next QK_q starts as soon as S_q is in registers, so it overlaps this tile's
-// softmax.
-// Tensor memory (512 columns): S_0, S_1 (128 fp32 columns each), O_0, O_1 (DP columns each),
-// and P_0, P_1 (bf16 pairs, 64 columns each) in their own columns when DP <= 64, otherwise over
-// the first half of S_q (then S_q is rewritten only after PV_q has consumed P_q).
-// Registers are rebalanced with setmaxnreg (RegSplit): producer/MMA 80, epilogue 48 (DP <= 64) or
-// 64 (80 when merging), softmax the rest (176-184).
+//   warp 12     TMA producer: Q (two tiles) per item, then K_j / V_j into a STAGES-deep ring; it
+//               also publishes each item's decoded plan (ItemPlan) to the other roles
+//   warps 13,14 MMA issuers, one thread per query tile: S_q = Q_q K_j^T (SS form), O_q += P_q V_j
+//               (TS form, P from tensor memory)
+// Both query tiles share every K/V tile (loaded once per 256 rows).  K/V tiles are 128 keys for
+// DP <= 64 and 64 keys for DP = 128, so that P always has its own tensor-memory columns: the
+// next QK_q starts as soon as the softmax holds S_q in registers, overlapping this tile's
+// softmax.  Tensor memory (512 columns): S_0, S_1 (BN fp32 columns each), P_0, P_1 (BN/2 columns
+// of bf16 pairs each), O_0, O_1 (DP columns each).  (With FmhaCfg's RA_D128_BN64 = 0, DP = 128
+// uses 128-key tiles with P written over S and one issuer in the fixed order PV_0(j), QK_0(j+1),
+// PV_1(j), QK_1(j+1); both layouts measure within 2 %.)
+// Registers are rebalanced with setmaxnreg (RegSplit) per instance, without spills in every
+// instance without a sliding window.
 // Hand-offs: an issuer polls every barrier an MMA group needs in one loop, the softmax tests its
-// next barriers while its exponentials run, and work-item index arithmetic uses launch-time
-// multiply-shift dividers (an integer divide would queue behind the exponentials on the MUFU).
-// The softmax arithmetic uses packed fp32x2 instructions and three-input max.  A polynomial
-// exp2 on the FMA pipe (exp2_poly3) can take 1 in kEmuEvery column pairs of unmasked tiles; it
-// is off by default (measured slower).
+// next barriers while its exponentials run (at DP = 128 the two softmax warpgroups take turns at
+// the exponential loop), and work-item index arithmetic uses launch-time multiply-shift dividers
+// (an integer divide would queue behind the exponentials on the MUFU).  The softmax arithmetic
+// uses packed fp32x2 instructions and three-input max.  A polynomial exp2 on the FMA pipe
+// (exp2_poly3) can take 1 in kEmuEvery column pairs of unmasked tiles; it is off by default
+// (measured slower).  A column-split softmax (RA_SOFTMAX_SPLIT) is off by default (measured
+// slower).
+// Programmatic dependent launch: each CTA signals dependents once set up; the epilogue waits for
+// any prerequisite grid before it touches memory (the next ring step's accumulator).
 // Every wait is bounded; on a timeout all roles stop, tensor memory is freed and the kernel
 // returns with the device status word set.
 #pragma once
