@@ -1,0 +1,39 @@
+"""The benchmark's JSON contract on the CPU: the reference arm (the fp64 oracle timed on the host
+cores) prints one line with the keys the GPU arm's line also carries."""
+
+import io
+import json
+import os
+import sys
+from contextlib import redirect_stdout
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_reference_arm_line():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        rc = bench.main(["--impl", "reference", "--config", "1", "--steps", "2", "--warmup", "3"])
+    assert rc == 0
+    lines = [ln for ln in buf.getvalue().splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["value"] > 0
+    assert d["config"]["workload"].startswith("cfg1")
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_bench_rejects_too_few_warmup_steps():
+    sys.path.insert(0, ROOT)
+    import bench
+    import pytest
+
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--config", "1", "--warmup", "2"])

@@ -71,3 +71,16 @@ def test_host_pipeline_against_the_oracle_and_pageable_memory(ra):
     o_p, l_p = _run_host(ra, q, k, v, 4, "striped", True, 3, pinned=False)
     assert torch.equal(o_p, o_h) and torch.equal(l_p, l_h)
     assert np.isfinite(to64(l_h)).all()
+
+
+def test_host_pipeline_without_lse(ra):
+    """lse_host and lse_dev both NULL: only O travels back, and it equals the device ring's."""
+    q, k, v = I.make_small(1, 4, 512, 64, "bf16", seed=5)
+    hq, hk, hv = (x.pin_memory() for x in (q, k, v))
+    o_h = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    dq, dk, dv, do = (torch.empty(x.shape, dtype=x.dtype, device="cuda") for x in (q, k, v, q))
+    streams = ra.ring_fwd_host(hq, hk, hv, 8, "contiguous", True, o_h, None, dq, dk, dv, do, None, n_chunks=2)
+    streams[1].synchronize()
+    o_ref, _ = ra.ring_attention(q.cuda(), k.cuda(), v.cuda(), 8, "contiguous", True, schedule="fused")
+    torch.cuda.synchronize()
+    assert torch.equal(o_h, o_ref.cpu())
