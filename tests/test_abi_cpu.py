@@ -173,3 +173,36 @@ def test_host_pipeline_validation(ra):
     assert call(lse_d=None) == ra.RA_ERR_INVALID_ARG and b"both" in lib.ra_last_error()
     assert call(st=same) == ra.RA_ERR_INVALID_ARG and b"distinct streams" in lib.ra_last_error()
     assert call(chunks=0) == ra.RA_ERR_INVALID_ARG and b"n_chunks" in lib.ra_last_error()
+
+
+def test_header_compiles_and_links_from_c(ra, tmp_path):
+    """The boundary as a C caller sees it: the header compiles as C and as C++, and a C program
+    that takes the address of every declared entry point links against the library and runs
+    (ra_version and ra_status_string need no device)."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    inc = os.path.join(ROOT, "include")
+    names = _declared_symbols()
+    src = tmp_path / "abi.c"
+    body = "\n".join(f"  fns[{i}] = (void (*)(void))&{n};" for i, n in enumerate(names))
+    src.write_text(
+        "#include <stdio.h>\n#include \"ra_attn.h\"\n"
+        f"int main(void) {{\n  void (*fns[{len(names)}])(void);\n{body}\n"
+        "  for (unsigned i = 0; i < sizeof(fns) / sizeof(fns[0]); ++i) if (!fns[i]) return 2;\n"
+        "  printf(\"%d %s\\n\", ra_version(), ra_status_string(RA_ERR_WORKSPACE));\n  return 0;\n}\n")
+    for lang, comp in (("c", gcc), ("c++", shutil.which("g++") or gcc)):
+        r = subprocess.run([comp, "-fsyntax-only", "-Wall", "-Werror", "-x", lang, os.path.join(inc, "ra_attn.h")],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, (lang, r.stderr)
+    libdir = os.path.dirname(ra.LIB_PATH)
+    exe = tmp_path / "abi"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-L", libdir, "-lra_attn",
+                        f"-Wl,-rpath,{libdir}", "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split() == [str(ra.version()), "RA_ERR_WORKSPACE"]
