@@ -37,3 +37,17 @@ def test_bench_rejects_too_few_warmup_steps():
 
     with pytest.raises(SystemExit):
         bench.main(["--impl", "reference", "--config", "1", "--warmup", "2"])
+
+
+def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
+    """Under torchrun every rank runs the reference arm's command; only rank 0 works and prints."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        rc = bench.main(["--impl", "reference", "--gpus", "2", "--config", "1", "--steps", "1", "--warmup", "3"])
+    assert rc == 0 and buf.getvalue().strip() == ""
