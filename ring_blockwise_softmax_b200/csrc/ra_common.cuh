@@ -362,6 +362,7 @@ __host__ __device__ __forceinline__ int fmod_(int n, const FastDiv& f) {
 struct AttnWork {
   int B;          // batch
   int r_major;    // work-item order: 1 = query shards outermost (contiguous shards), 0 = blocks
+  int tile_major; // K/V walk of a multi-step launch: 1 = tile index outermost, the shards inside
   int hgroup;     // heads per item group (the group's K/V is sized to stay resident in L2)
   int n_q;        // query tokens per shard
   int n_kv;       // key tokens per shard

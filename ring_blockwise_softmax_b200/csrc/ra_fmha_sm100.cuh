@@ -356,11 +356,37 @@ __device__ __forceinline__ void decode_item(const AttnWork& w, int idx, Item& it
   it.pos_first = it.pos0 + static_cast<long long>(it.t0) * w.q_tstride;
 }
 
+// Striped shards (shard s holds the keys at positions u * P + s): for a position D = a * P + b
+// (0 <= b < P), the keys of shard s at or before D are u <= a - (s > b), and the keys at or after
+// D are u >= a + (b > s).  Launches with a tile-major walk have exactly this geometry, so their
+// per-tile bounds need no division.
+struct StripedPos {
+  int a, b;  // b = -1: a position before the first key (every key is at or after it)
+};
+__device__ __forceinline__ StripedPos striped_pos(const AttnWork& w, long long pos) {
+  if (pos < 0) return {0, -1};
+  const int a = pos < 0x7fffffffLL ? fdiv(static_cast<int>(pos), w.fd_P) : static_cast<int>(pos / w.P);
+  return {a, static_cast<int>(pos - static_cast<long long>(a) * w.P)};
+}
+// visible_key_limit for a query at p (causal bound; all keys otherwise).
+__device__ __forceinline__ int striped_lim(const AttnWork& w, StripedPos p, int s) {
+  if (!w.causal) return w.n_kv;
+  return min(w.n_kv, p.a + 1 - (s > p.b ? 1 : 0));
+}
+// visible_key_start for a window whose first position is p.
+__device__ __forceinline__ int striped_start(const AttnWork& w, StripedPos p, int s) {
+  return min(w.n_kv, p.a + (p.b > s ? 1 : 0));
+}
+
 struct Walk {
   int step;  // ring step offset within this launch
   int s;     // KV shard
   int u0;    // first key of the current tile
   int lim;   // keys of shard s visible to the item's last row
+  // Tile-major walk: the largest lim over the launch's shards, the shard of step 0, and the
+  // item's last position and first window position.
+  int umax, s0;
+  StripedPos last, first;
 };
 
 // Keys [start, lim) of shard s are visible to some row of the item: lim from its last row (the
@@ -383,14 +409,65 @@ __device__ __forceinline__ bool walk_seek(Walk& k, const AttnWork& w, const Item
   return false;
 }
 
+// The tile-major walk is compiled into the 64-key-tile (d = 128) kernels only: the 128-key-tile
+// kernels keep their registers for the softmax (their ring workloads use contiguous shards).
+template <int BN>
+constexpr bool kTileWalk = BN == 64;
+
+// Tile-major order (w.tile_major, striped shards): tile u0 of every shard that has it, then tile
+// u0 + BN, ...  Striped shards interleave their keys in memory, so this order reads each stretch
+// of K/V once per item instead of once per shard.  Same tiles as the shard-major walk.
+template <bool WIN, int BN>
+__device__ __forceinline__ bool walk_seek_tiles(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
+  while (k.u0 < k.umax) {
+    for (; k.step < n_steps; ++k.step) {
+      int s = k.s0 - k.step;
+      while (s < 0) s += w.P;
+      const int lim = striped_lim(w, k.last, s);
+      const int start = WIN ? striped_start(w, k.first, s) : 0;
+      if (lim > start && k.u0 < lim && k.u0 + BN > start) {
+        k.s = s;
+        k.lim = lim;
+        return true;
+      }
+    }
+    k.step = 0;
+    k.u0 += BN;
+  }
+  return false;
+}
+
 template <bool WIN, int BN>
 __device__ __forceinline__ bool walk_begin(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
   k.step = 0;
+  if (kTileWalk<BN> && w.tile_major) {
+    k.s0 = ring_shard(w, it.r, w.ring_step);
+    k.last = striped_pos(w, it.pos_last);
+    k.first = (WIN && w.window > 0) ? striped_pos(w, it.pos_first - w.window + 1) : StripedPos{0, -1};
+    int umax = 0, ulo = 0x7fffffff;
+    for (int step = 0; step < n_steps; ++step) {
+      int s = k.s0 - step;
+      while (s < 0) s += w.P;
+      const int lim = striped_lim(w, k.last, s);
+      const int start = WIN ? striped_start(w, k.first, s) : 0;
+      if (lim > start) {
+        umax = max(umax, lim);
+        ulo = min(ulo, start & ~(BN - 1));
+      }
+    }
+    k.umax = umax;
+    k.u0 = umax > 0 ? ulo : 0;
+    return walk_seek_tiles<WIN, BN>(k, w, it, n_steps);
+  }
   return walk_seek<WIN, BN>(k, w, it, n_steps);
 }
 
 template <bool WIN, int BN>
 __device__ __forceinline__ bool walk_next(Walk& k, const AttnWork& w, const Item& it, int n_steps) {
+  if (kTileWalk<BN> && w.tile_major) {
+    ++k.step;
+    return walk_seek_tiles<WIN, BN>(k, w, it, n_steps);
+  }
   k.u0 += BN;
   if (k.u0 < k.lim) return true;
   ++k.step;
@@ -1221,11 +1298,21 @@ __global__ void __launch_bounds__(FmhaCfg<DP>::THREADS, 1)
       float l_sum = 0.f;         // running sum of 2^(x - m_used)
       Walk wk;
       int cur_s = -1, row_lim = 0, row_lo = 0;
+      StripedPos row_last{0, -1}, row_first{0, -1};  // tile-major launches: this row's position and window start
+      if (kTileWalk<C::BN> && w.tile_major) {
+        row_last = striped_pos(w, pos_q);
+        if (WIN && w.window > 0) row_first = striped_pos(w, pos_q - w.window + 1);
+      }
       for (bool has = walk_begin<WIN, C::BN>(wk, w, it, n_steps); has; has = walk_next<WIN, C::BN>(wk, w, it, n_steps)) {
         if (wk.s != cur_s) {
           cur_s = wk.s;
-          row_lim = row_ok ? visible_key_limit(w, pos_q, wk.s) : w.n_kv;
-          if (WIN) row_lo = row_ok ? visible_key_start(w, pos_q, wk.s) : 0;
+          if (kTileWalk<C::BN> && w.tile_major) {
+            row_lim = row_ok ? striped_lim(w, row_last, wk.s) : w.n_kv;
+            if (WIN) row_lo = row_ok ? striped_start(w, row_first, wk.s) : 0;
+          } else {
+            row_lim = row_ok ? visible_key_limit(w, pos_q, wk.s) : w.n_kv;
+            if (WIN) row_lo = row_ok ? visible_key_start(w, pos_q, wk.s) : 0;
+          }
         }
         if (!__all_sync(0xffffffffu, s_seen)) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + q, c & 1, ctl, 0x301));

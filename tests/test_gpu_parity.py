@@ -161,6 +161,21 @@ def test_lse_merge_n(ra, d, k):
 
 # ------------------------------------------------------------------------------- ring driver
 
+@pytest.mark.parametrize("P,N", [(2, 600), (3, 384), (8, 1000), (16, 1040)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("schedule", ["stepwise", "fused"])
+def test_ring_striped_d128(ra, P, N, causal, schedule):
+    """Striped rings at d = 128, whose fused launches walk K/V tile index first and the shards
+    inside (shards of 300, 128, 125 and 65 rows: ragged 64-key tiles in every shard)."""
+    q, k, v = I.make_small(1, 2, N, 128, "bf16", seed=31 * P + N)
+    qd, kd, vd = _dev(q, k, v)
+    o, lse = ra.ring_attention(qd, kd, vd, P, "striped", causal, schedule=schedule)
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == ra.RA_OK
+    o_ref, l_ref = oracle_heads(to64(q), to64(k), to64(v), 1 / math.sqrt(128), causal)
+    compare(to64(o), to64(lse), o_ref, l_ref, "bf16", f"striped d=128 P={P} causal={causal} {schedule}")
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("layout", ["contiguous", "striped"])
 @pytest.mark.parametrize("causal", [False, True])

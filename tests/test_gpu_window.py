@@ -51,14 +51,15 @@ def test_window_wider_than_the_sequence_is_causal(ra):
 @pytest.mark.parametrize("layout", ["contiguous", "striped"])
 @pytest.mark.parametrize("schedule", ["stepwise", "fused"])
 @pytest.mark.parametrize("window", [100, 300])
-def test_window_ring(ra, layout, schedule, window):
-    B, H, N, d, P = 1, 2, 1024, 64, 4
-    q, k, v = I.make_small(B, H, N, d, "bf16", seed=2200 + window, v_dist="uniform")
+@pytest.mark.parametrize("d", [64, 128])
+def test_window_ring(ra, layout, schedule, window, d):
+    B, H, N, P = 1, 2, 1024, 4
+    q, k, v = I.make_small(B, H, N, d, "bf16", seed=2200 + window + d, v_dist="uniform")
     qd, kd, vd = _dev(q, k, v)
     o, lse = ra.ring_attention(qd, kd, vd, P, layout, True, schedule=schedule, window=window)
     torch.cuda.synchronize()
-    o_ref, l_ref = oracle_heads(to64(q), to64(k), to64(v), 1 / 8, True, window=window)
-    compare(to64(o), to64(lse), o_ref, l_ref, "bf16", f"window ring {layout} {schedule} w={window}")
+    o_ref, l_ref = oracle_heads(to64(q), to64(k), to64(v), 1 / math.sqrt(d), True, window=window)
+    compare(to64(o), to64(lse), o_ref, l_ref, "bf16", f"window ring {layout} {schedule} w={window} d={d}")
     o1, l1 = ra.attention(qd, kd, vd, window=window)
     torch.cuda.synchronize()
     compare(to64(o), to64(lse), to64(o1), to64(l1), "bf16", "window ring vs single pass")
