@@ -26,13 +26,15 @@
 // S and dP here are the transposes of each other's roles in the two instances, so both use the
 // forward's operand forms unchanged.  No atomics: every gradient element has one owner.
 //
-// Roles (320 threads): two element-wise warpgroups (warps 0-3 and 4-7) take alternate streamed
+// Roles (352 threads): two element-wise warpgroups (warps 0-3 and 4-7) take alternate streamed
 // tiles, thread = tensor-memory lane (warp % 4) * 32 + lane, all 64 columns of its row; each
 // warpgroup has its own (S, dP) buffer and P, dS columns in tensor memory, so one computes while
 // the other waits on its loads, stores and barriers.  (The dK/dV instance at DP = 128 lacks the
-// tensor memory for that and runs attn_bwd_sm100_split, further below.)  Warp 8 is the TMA producer (and allocates
-// tensor memory), warp 9 the MMA issuer: it starts S, dP of tile j + 2 as soon as warpgroup j % 2
-// holds tile j in registers.  At the end the eight warps run the epilogue.  Every wait is bounded.
+// tensor memory for that and runs attn_bwd_sm100_split, further below.)  Warp 8 is the TMA
+// producer (and allocates tensor memory); warps 9 and 10 issue the MMAs: warp 9 starts S, dP of
+// tile j + 2 as soon as warpgroup j % 2 holds tile j in registers, warp 10 the products of each
+// tile once its P and dS are stored.  At the end the eight warps run the epilogue.  Every wait is
+// bounded.
 #pragma once
 
 #include "ra_common.cuh"
@@ -103,7 +105,7 @@ struct BwdCfg {
   static constexpr int BAR_BYTES = (NBAR * 8 + 15) / 16 * 16;
   // + tensor-memory slot and abort flag (16 B) + statistics [2 warpgroups][2 slots][BN] float2.
   static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + BAR_BYTES + 16 + 4 * BN * 8;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;
 };
 
 // The streamed tiles of one CTA: tiles tb .. te-1 (of BN rows) of each of `heads` streamed heads.
@@ -204,7 +206,7 @@ __device__ __forceinline__ void bwd_drain(uint64_t* bar, uint32_t parity, uint64
 }
 
 template <int DP, bool KV>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_bwd_sm100(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
                    const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
                    const __grid_constant__ CUtensorMap tm_b3, const BwdTcWork w) {
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar_p_full + i, 4);
       mbar_init(bar_pv_done + i, 1);
     }
-    mbar_init(bar_acc_done, 1);
+    mbar_init(bar_acc_done, 2);  // one commit per issuer
     for (int i = 0; i < 4; ++i) mbar_init(bar_stats + i, 4);
     *abort_flag = 0;
     fence_mbar_init();
@@ -308,9 +310,12 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = (j > C::STAGES ? j - C::STAGES : 0); i < j; ++i)
         bwd_drain(bar_stage_full + i % C::STAGES, (i / C::STAGES) & 1, w.wait_limit_ns);
     }
-  } else if (warp == 9) {
+  } else if (warp == 9 || warp == 10) {
     if (lane == 0) {
-      // ================================================================ MMA issuer
+      // ================================================================ MMA issuers
+      // Two issuing threads (warp 9: S and dP; warp 10: the gradient products): one thread issues
+      // a tcgen05.mma about every 115 cycles whatever its size, which for these 128 x 64 x 16 and
+      // 128 x d x 16 shapes is far below the tensor core's rate, so a second issuer doubles it.
       constexpr uint32_t idesc_s = make_idesc_bf16(128, C::BN, 0, 0);
       constexpr uint32_t idesc_acc = make_idesc_bf16(128, DP, 0, 1);
       const uint64_t kmaj = make_smem_desc(0, 16, C::ATOM_BYTES, C::SWZ);
@@ -360,16 +365,18 @@ __global__ void __launch_bounds__(320, 1)
         mma_commit(bar_stage_empty + sp);
         return true;
       };
-      bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
-      if (ok) ok = issue_s(0);
-      if (ok && rg.n > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < rg.n; ++j) {
-        // S(j + 2) first: it only needs warpgroup j % 2 to hold S(j), so it runs while that
-        // warpgroup computes tile j.
-        if (j + 2 < rg.n && !issue_s(j + 2)) break;
-        if (!issue_acc(j)) break;
+      if (warp == 9) {
+        // S, dP of every tile, each as soon as its stage has landed and its warpgroup holds the
+        // tile two before it in registers.
+        bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
+        for (int j = 0; ok && j < rg.n; ++j) ok = issue_s(j);
+      } else {
+        // The products of every tile, as soon as its P and dS are in tensor memory.
+        bool ok = rg.n > 0;
+        for (int j = 0; ok && j < rg.n; ++j) ok = issue_acc(j);
       }
-      // The epilogue waits on acc_done: every MMA issued has completed (also after an abort).
+      // The epilogue waits on acc_done: every MMA either issuer issued has completed (also after
+      // an abort).
       if (rg.n > 0)
         mma_commit(bar_acc_done);
       else
@@ -636,11 +643,11 @@ struct BwdCfgSplit {
   static constexpr int NBAR = 1 + 2 * STAGES + 7 + 2;
   static_assert((NBAR * 8) % 16 == 0, "statistics buffer must stay 16-byte aligned");
   static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + NBAR * 8 + 16 + 4 * BN * 4;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;
 };
 
 template <int DP, bool KV>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_bwd_sm100_split(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
                    const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
                    const __grid_constant__ CUtensorMap tm_b3, const BwdTcWork w) {
@@ -682,7 +689,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(bar_p_full, 8);
     mbar_init(bar_pv_done, 1);
-    mbar_init(bar_acc_done, 1);
+    mbar_init(bar_acc_done, 2);  // one commit per issuer
     mbar_init(bar_stats + 0, 8);
     mbar_init(bar_stats + 1, 8);
     *abort_flag = 0;
@@ -745,9 +752,12 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = (j > C::STAGES ? j - C::STAGES : 0); i < j; ++i)
         bwd_drain(bar_stage_full + i % C::STAGES, (i / C::STAGES) & 1, w.wait_limit_ns);
     }
-  } else if (warp == 9) {
+  } else if (warp == 9 || warp == 10) {
     if (lane == 0) {
-      // ================================================================ MMA issuer
+      // ================================================================ MMA issuers
+      // Two issuing threads (warp 9: S and dP; warp 10: the gradient products): one thread issues
+      // a tcgen05.mma about every 115 cycles whatever its size, which for these 128 x 64 x 16 and
+      // 128 x d x 16 shapes is far below the tensor core's rate, so a second issuer doubles it.
       constexpr uint32_t idesc_s = make_idesc_bf16(128, C::BN, 0, 0);
       constexpr uint32_t idesc_acc = make_idesc_bf16(128, DP, 0, 1);
       const uint64_t kmaj = make_smem_desc(0, 16, C::ATOM_BYTES, C::SWZ);
@@ -796,23 +806,18 @@ __global__ void __launch_bounds__(320, 1)
         mma_commit(bar_stage_empty + sp);
         return true;
       };
-      bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
-      if (C::NSB == 1) {
-        // S(j + 1) as soon as S(j) is in registers, then the products of tile j.
-        for (int j = 0; ok && j <= rg.n; ++j) {
-          if (j < rg.n && !issue_s(j)) break;
-          if (j > 0 && !issue_acc(j - 1)) break;
-        }
+      if (warp == 9) {
+        // S, dP of every tile, each as soon as its stage has landed and the element-wise warps
+        // hold the previous tile of its buffer in registers.
+        bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
+        for (int j = 0; ok && j < rg.n; ++j) ok = issue_s(j);
       } else {
-        // Two tiles ahead: S(j + 2) right after the products of tile j.
-        if (ok) ok = issue_s(0);
-        if (ok && rg.n > 1) ok = issue_s(1);
-        for (int j = 0; ok && j < rg.n; ++j) {
-          if (!issue_acc(j)) break;
-          if (j + 2 < rg.n && !issue_s(j + 2)) break;
-        }
+        // The products of every tile, as soon as its P and dS are in tensor memory.
+        bool ok = rg.n > 0;
+        for (int j = 0; ok && j < rg.n; ++j) ok = issue_acc(j);
       }
-      // The epilogue waits on acc_done: every MMA issued has completed (also after an abort).
+      // The epilogue waits on acc_done: every MMA either issuer issued has completed (also after
+      // an abort).
       if (rg.n > 0)
         mma_commit(bar_acc_done);
       else
