@@ -21,6 +21,13 @@ static cudaError_t launch_kernel(K kern, bool kv, const CUtensorMap& a1, const C
                                  cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
+  // The kernel's warpgroups rebalance registers with setmaxnreg; an increase beyond the pool the
+  // block was launched with would never complete, so such a build is refused here.
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs * C::THREADS < C::REG_TOTAL || attr.maxThreadsPerBlock < C::THREADS)
+    return cudaErrorInvalidConfiguration;
   const int rows = kv ? w.n_kv : w.n_q;
   const dim3 grid((rows + C::BM - 1) / C::BM, kv ? w.H_kv : w.H, w.B);
   if (!(kv && RA_PDL)) {

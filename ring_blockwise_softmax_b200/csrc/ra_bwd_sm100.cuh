@@ -105,7 +105,14 @@ struct BwdCfg {
   static constexpr int BAR_BYTES = (NBAR * 8 + 15) / 16 * 16;
   // + tensor-memory slot and abort flag (16 B) + statistics [2 warpgroups][2 slots][BN] float2.
   static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + BAR_BYTES + 16 + 4 * BN * 8;
-  static constexpr int THREADS = 352;
+  static constexpr int THREADS = 384;
+  // Registers: at launch 65536 / THREADS (rounded down to 8) for every thread; the control
+  // warpgroup (producer and issuers) gives up all but REG_CTL to the element-wise warpgroups.
+  static constexpr int REG_LAUNCH = (65536 / THREADS) / 8 * 8;
+  static constexpr int REG_CTL = 96;
+  static constexpr int REG_EW = ((REG_LAUNCH * THREADS - 128 * REG_CTL) / 256) / 8 * 8;
+  static constexpr int REG_TOTAL = 256 * REG_EW + 128 * REG_CTL;
+  static_assert(REG_TOTAL <= REG_LAUNCH * THREADS, "register split exceeds the launch");
 };
 
 // The streamed tiles of one CTA: tiles tb .. te-1 (of BN rows) of each of `heads` streamed heads.
@@ -165,6 +172,18 @@ __device__ __forceinline__ BwdRange bwd_range(const BwdTcWork& w) {
   return r;
 }
 
+// Warpgroup-wide register reallocation (every warp of the warpgroup executes it).  An increase
+// waits until the block's register pool, fixed at launch, has the registers free: the host checks
+// the compiled kernel's pool against the split before every launch.
+template <int N>
+__device__ __forceinline__ void bwd_setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void bwd_setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // low 16 bits = lo
   return *reinterpret_cast<uint32_t*>(&v);
@@ -206,7 +225,7 @@ __device__ __forceinline__ void bwd_drain(uint64_t* bar, uint32_t parity, uint64
 }
 
 template <int DP, bool KV>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_bwd_sm100(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
                    const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
                    const __grid_constant__ CUtensorMap tm_b3, const BwdTcWork w) {
@@ -243,12 +262,12 @@ __global__ void __launch_bounds__(352, 1)
       mbar_init(bar_stage_empty + i, KV ? 1 + 4 : 1);  // MMA commit (+ the 4 warps reading O)
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_s_full + i, 1);
+      mbar_init(bar_s_full + i, 2);  // the S and the dP issuer
       mbar_init(bar_s_free + i, 4);  // one arrival per warp of the warpgroup
       mbar_init(bar_p_full + i, 4);
       mbar_init(bar_pv_done + i, 1);
     }
-    mbar_init(bar_acc_done, 2);  // one commit per issuer
+    mbar_init(bar_acc_done, 3);  // one commit per issuer
     for (int i = 0; i < 4; ++i) mbar_init(bar_stats + i, 4);
     *abort_flag = 0;
     fence_mbar_init();
@@ -274,8 +293,11 @@ __global__ void __launch_bounds__(352, 1)
   // end.  Every CTA waits for any such prerequisite grid before it exits (below), so neither
   // launch completes before the one ahead of it on the stream.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-  if (warp == 8) {
+  // Register split (warpgroup-wide): the control warpgroup (warps 8-11) shrinks, and the
+  // element-wise warpgroups grow into what it released.
+  if (warp >= 8) {
+   bwd_setmaxnreg_dec<C::REG_CTL>();
+   if (warp == 8) {
     if (lane == 0 && rg.n > 0) {
       // ================================================================ TMA producer
       mbar_arrive_expect_tx(bar_fixed, 2 * C::FIX_BYTES);
@@ -310,12 +332,13 @@ __global__ void __launch_bounds__(352, 1)
       for (int i = (j > C::STAGES ? j - C::STAGES : 0); i < j; ++i)
         bwd_drain(bar_stage_full + i % C::STAGES, (i / C::STAGES) & 1, w.wait_limit_ns);
     }
-  } else if (warp == 9 || warp == 10) {
+   } else {
     if (lane == 0) {
       // ================================================================ MMA issuers
-      // Two issuing threads (warp 9: S and dP; warp 10: the gradient products): one thread issues
-      // a tcgen05.mma about every 115 cycles whatever its size, which for these 128 x 64 x 16 and
-      // 128 x d x 16 shapes is far below the tensor core's rate, so a second issuer doubles it.
+      // Three issuing threads (warp 9: S, warp 10: dP, warp 11: the gradient products): one
+      // thread issues a tcgen05.mma about every 115 cycles whatever its size, far below the tensor
+      // core's rate for these 128 x 64 x 16 and 128 x d x 16 shapes, so the MMA rate grows with
+      // the number of issuing threads.
       constexpr uint32_t idesc_s = make_idesc_bf16(128, C::BN, 0, 0);
       constexpr uint32_t idesc_acc = make_idesc_bf16(128, DP, 0, 1);
       const uint64_t kmaj = make_smem_desc(0, 16, C::ATOM_BYTES, C::SWZ);
@@ -330,17 +353,17 @@ __global__ void __launch_bounds__(352, 1)
                        ((jj >> 1) - 1) & 1, ctl, 0x712))
           return false;
         tc_fence_after();
-        const uint32_t b1 = stage0 + st * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
-        const uint64_t da1 = kmaj | ((a1 >> 4) & 0x3FFFu), da2 = kmaj | ((a2 >> 4) & 0x3FFFu);
-        const uint64_t db1 = kmaj | ((b1 >> 4) & 0x3FFFu), db2 = kmaj | ((b2 >> 4) & 0x3FFFu);
-        const uint32_t col = tmem + b * C::SB_STRIDE;
+        // S = A1 B1^T (warp 9) or dP = A2 B2^T (warp 10); s_full completes on both commits.
+        const uint32_t bx = stage0 + st * C::STAGE_BYTES + (warp == 9 ? 0 : C::TILE_BYTES);
+        const uint32_t ax = warp == 9 ? a1 : a2;
+        const uint64_t da = kmaj | ((ax >> 4) & 0x3FFFu), dbx = kmaj | ((bx >> 4) & 0x3FFFu);
+        const uint32_t col = tmem + b * C::SB_STRIDE + (warp == 9 ? C::S_COL : C::DP_COL);
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk) {
           const int cb = (kk * 16) / C::CB;
           const uint32_t in = ((kk * 16) % C::CB) * 2;
           const uint32_t offa = (cb * C::BLK_M + in) >> 4, offb = (cb * C::BLK_N + in) >> 4;
-          mma_ss(col + C::S_COL, da1 + offa, db1 + offb, idesc_s, kk > 0 ? 1u : 0u);
-          mma_ss(col + C::DP_COL, da2 + offa, db2 + offb, idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(col, da + offa, dbx + offb, idesc_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_s_full + b);
         return true;
@@ -365,8 +388,8 @@ __global__ void __launch_bounds__(352, 1)
         mma_commit(bar_stage_empty + sp);
         return true;
       };
-      if (warp == 9) {
-        // S, dP of every tile, each as soon as its stage has landed and its warpgroup holds the
+      if (warp == 9 || warp == 10) {
+        // S (dP) of every tile, each as soon as its stage has landed and its warpgroup holds the
         // tile two before it in registers.
         bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
         for (int j = 0; ok && j < rg.n; ++j) ok = issue_s(j);
@@ -383,7 +406,9 @@ __global__ void __launch_bounds__(352, 1)
         mbar_arrive(bar_acc_done);
       bwd_drain(bar_acc_done, 0, w.wait_limit_ns);
     }
+   }
   } else {
+    bwd_setmaxnreg_inc<C::REG_EW>();
     // ==================================================================== element-wise (warps 0-7)
     const int grp = warp >> 2;  // warpgroup: streamed tiles j with j % 2 == grp
     const int row = (warp & 3) * 32 + lane;
@@ -490,6 +515,13 @@ __global__ void __launch_bounds__(352, 1)
         uint32_t sv[32], pv[32];
         tmem_ld32(sbuf + C::S_COL + 32 * h, sv);
         tmem_ld32(sbuf + C::DP_COL + 32 * h, pv);
+        // The columns' (LSE log2(e), D) pairs (dK/dV instance), read from shared memory while the
+        // tensor-memory loads are in flight rather than one by one at their uses.
+        float4 cst[16];
+        if (KV) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) cst[i] = stv[16 * h + i];
+        }
         tmem_ld_wait(sv);
         reg_pin32(pv);
         if (h == 1) {
@@ -524,7 +556,7 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           float4 cs = make_float4(row_l2, row_d, row_l2, row_d);  // (LSE log2(e), D) of columns i, i + 1
-          if (KV) cs = stv[16 * h + i / 2];
+          if (KV) cs = cst[i / 2];
           float e0 = bwd_ex2(fmaf(__uint_as_float(sv[i]), w.scale_log2, -cs.x));
           float e1 = bwd_ex2(fmaf(__uint_as_float(sv[i + 1]), w.scale_log2, -cs.z));
           if (masked) {
@@ -643,11 +675,18 @@ struct BwdCfgSplit {
   static constexpr int NBAR = 1 + 2 * STAGES + 7 + 2;
   static_assert((NBAR * 8) % 16 == 0, "statistics buffer must stay 16-byte aligned");
   static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + NBAR * 8 + 16 + 4 * BN * 4;
-  static constexpr int THREADS = 352;
+  static constexpr int THREADS = 384;
+  // Registers: at launch 65536 / THREADS (rounded down to 8) for every thread; the control
+  // warpgroup (producer and issuers) gives up all but REG_CTL to the element-wise warpgroups.
+  static constexpr int REG_LAUNCH = (65536 / THREADS) / 8 * 8;
+  static constexpr int REG_CTL = 96;
+  static constexpr int REG_EW = ((REG_LAUNCH * THREADS - 128 * REG_CTL) / 256) / 8 * 8;
+  static constexpr int REG_TOTAL = 256 * REG_EW + 128 * REG_CTL;
+  static_assert(REG_TOTAL <= REG_LAUNCH * THREADS, "register split exceeds the launch");
 };
 
 template <int DP, bool KV>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_bwd_sm100_split(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
                    const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
                    const __grid_constant__ CUtensorMap tm_b3, const BwdTcWork w) {
@@ -684,12 +723,12 @@ __global__ void __launch_bounds__(352, 1)
       mbar_init(bar_stage_empty + i, KV ? 1 + 8 : 1);  // MMA commit (+ the 8 warps reading O)
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_s_full + i, 1);
+      mbar_init(bar_s_full + i, 2);  // the S and the dP issuer
       mbar_init(bar_s_free + i, 8);  // one arrival per element-wise warp
     }
     mbar_init(bar_p_full, 8);
     mbar_init(bar_pv_done, 1);
-    mbar_init(bar_acc_done, 2);  // one commit per issuer
+    mbar_init(bar_acc_done, 3);  // one commit per issuer
     mbar_init(bar_stats + 0, 8);
     mbar_init(bar_stats + 1, 8);
     *abort_flag = 0;
@@ -716,8 +755,11 @@ __global__ void __launch_bounds__(352, 1)
   // end.  Every CTA waits for any such prerequisite grid before it exits (below), so neither
   // launch completes before the one ahead of it on the stream.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-  if (warp == 8) {
+  // Register split (warpgroup-wide): the control warpgroup (warps 8-11) shrinks, and the
+  // element-wise warpgroups grow into what it released.
+  if (warp >= 8) {
+   bwd_setmaxnreg_dec<C::REG_CTL>();
+   if (warp == 8) {
     if (lane == 0 && rg.n > 0) {
       // ================================================================ TMA producer
       mbar_arrive_expect_tx(bar_fixed, 2 * C::FIX_BYTES);
@@ -752,12 +794,13 @@ __global__ void __launch_bounds__(352, 1)
       for (int i = (j > C::STAGES ? j - C::STAGES : 0); i < j; ++i)
         bwd_drain(bar_stage_full + i % C::STAGES, (i / C::STAGES) & 1, w.wait_limit_ns);
     }
-  } else if (warp == 9 || warp == 10) {
+   } else {
     if (lane == 0) {
       // ================================================================ MMA issuers
-      // Two issuing threads (warp 9: S and dP; warp 10: the gradient products): one thread issues
-      // a tcgen05.mma about every 115 cycles whatever its size, which for these 128 x 64 x 16 and
-      // 128 x d x 16 shapes is far below the tensor core's rate, so a second issuer doubles it.
+      // Three issuing threads (warp 9: S, warp 10: dP, warp 11: the gradient products): one
+      // thread issues a tcgen05.mma about every 115 cycles whatever its size, far below the tensor
+      // core's rate for these 128 x 64 x 16 and 128 x d x 16 shapes, so the MMA rate grows with
+      // the number of issuing threads.
       constexpr uint32_t idesc_s = make_idesc_bf16(128, C::BN, 0, 0);
       constexpr uint32_t idesc_acc = make_idesc_bf16(128, DP, 0, 1);
       const uint64_t kmaj = make_smem_desc(0, 16, C::ATOM_BYTES, C::SWZ);
@@ -772,17 +815,17 @@ __global__ void __launch_bounds__(352, 1)
                        ((jj / C::NSB) - 1) & 1, ctl, 0x712))
           return false;
         tc_fence_after();
-        const uint32_t b1 = stage0 + st * C::STAGE_BYTES, b2 = b1 + C::TILE_BYTES;
-        const uint64_t da1 = kmaj | ((a1 >> 4) & 0x3FFFu), da2 = kmaj | ((a2 >> 4) & 0x3FFFu);
-        const uint64_t db1 = kmaj | ((b1 >> 4) & 0x3FFFu), db2 = kmaj | ((b2 >> 4) & 0x3FFFu);
-        const uint32_t col = tmem + b * C::SB_STRIDE;
+        // S = A1 B1^T (warp 9) or dP = A2 B2^T (warp 10); s_full completes on both commits.
+        const uint32_t bx = stage0 + st * C::STAGE_BYTES + (warp == 9 ? 0 : C::TILE_BYTES);
+        const uint32_t ax = warp == 9 ? a1 : a2;
+        const uint64_t da = kmaj | ((ax >> 4) & 0x3FFFu), dbx = kmaj | ((bx >> 4) & 0x3FFFu);
+        const uint32_t col = tmem + b * C::SB_STRIDE + (warp == 9 ? C::S_COL : C::DP_COL);
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk) {
           const int cb = (kk * 16) / C::CB;
           const uint32_t in = ((kk * 16) % C::CB) * 2;
           const uint32_t offa = (cb * C::BLK_M + in) >> 4, offb = (cb * C::BLK_N + in) >> 4;
-          mma_ss(col + C::S_COL, da1 + offa, db1 + offb, idesc_s, kk > 0 ? 1u : 0u);
-          mma_ss(col + C::DP_COL, da2 + offa, db2 + offb, idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(col, da + offa, dbx + offb, idesc_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_s_full + b);
         return true;
@@ -806,8 +849,8 @@ __global__ void __launch_bounds__(352, 1)
         mma_commit(bar_stage_empty + sp);
         return true;
       };
-      if (warp == 9) {
-        // S, dP of every tile, each as soon as its stage has landed and the element-wise warps
+      if (warp == 9 || warp == 10) {
+        // S (dP) of every tile, each as soon as its stage has landed and the element-wise warps
         // hold the previous tile of its buffer in registers.
         bool ok = rg.n > 0 && mbar_wait(bar_fixed, 0, ctl, 0x711);
         for (int j = 0; ok && j < rg.n; ++j) ok = issue_s(j);
@@ -824,7 +867,9 @@ __global__ void __launch_bounds__(352, 1)
         mbar_arrive(bar_acc_done);
       bwd_drain(bar_acc_done, 0, w.wait_limit_ns);
     }
+   }
   } else {
+    bwd_setmaxnreg_inc<C::REG_EW>();
     // ==================================================================== element-wise (warps 0-7)
     const int grp = warp >> 2;           // 0: columns 0-31, 1: columns 32-63
     const int row = (warp & 3) * 32 + lane;
