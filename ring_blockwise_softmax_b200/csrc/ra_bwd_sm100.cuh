@@ -100,18 +100,24 @@ struct BwdCfg {
   // loaded while tile j's is still held: three stages.
   static_assert(STAGES >= 3, "the look-ahead needs a third stage");
   // Barriers: fixed_full, stage_full[S], stage_empty[S], s_full[2], s_free[2], p_full[2],
-  // pv_done[2], acc_done, stats[2][2] (per warpgroup and slot).
-  static constexpr int NBAR = 1 + 2 * STAGES + 8 + 1 + 4;
+  // pv_done[2], acc_done, stats_ready[4], stats_free[4] (per statistics slot).
+  static constexpr int NSLOT = 4;  // statistics slots: tile j uses slot j % NSLOT
+  static constexpr int NBAR = 1 + 2 * STAGES + 8 + 1 + 2 * NSLOT;
   static constexpr int BAR_BYTES = (NBAR * 8 + 15) / 16 * 16;
-  // + tensor-memory slot and abort flag (16 B) + statistics [2 warpgroups][2 slots][BN] float2.
-  static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + BAR_BYTES + 16 + 4 * BN * 8;
-  static constexpr int THREADS = 384;
+  // + tensor-memory slot and abort flag (16 B) + statistics [NSLOT][BN] float2.
+  static constexpr int SMEM_BYTES = 1024 + 2 * FIX_BYTES + STAGES * STAGE_BYTES + BAR_BYTES + 16 + NSLOT * BN * 8;
+  // The dK/dV instance has a fourth warpgroup (warps 12-15) that computes the streamed rows'
+  // statistics (LSE, D) ahead of the element-wise warps.
+  static constexpr bool STATS_WG = KV;
+  static constexpr int THREADS = STATS_WG ? 512 : 384;
   // Registers: at launch 65536 / THREADS (rounded down to 8) for every thread; the control
-  // warpgroup (producer and issuers) gives up all but REG_CTL to the element-wise warpgroups.
+  // warpgroup (producer and issuers) keeps REG_CTL, the statistics warpgroup REG_ST, and the
+  // element-wise warpgroups take the rest.
   static constexpr int REG_LAUNCH = (65536 / THREADS) / 8 * 8;
   static constexpr int REG_CTL = 96;
-  static constexpr int REG_EW = ((REG_LAUNCH * THREADS - 128 * REG_CTL) / 256) / 8 * 8;
-  static constexpr int REG_TOTAL = 256 * REG_EW + 128 * REG_CTL;
+  static constexpr int REG_ST = 40;
+  static constexpr int REG_EW = ((REG_LAUNCH * THREADS - 128 * REG_CTL - (STATS_WG ? 128 * REG_ST : 0)) / 256) / 8 * 8;
+  static constexpr int REG_TOTAL = 256 * REG_EW + 128 * REG_CTL + (STATS_WG ? 128 * REG_ST : 0);
   static_assert(REG_TOTAL <= REG_LAUNCH * THREADS, "register split exceeds the launch");
 };
 
@@ -225,7 +231,7 @@ __device__ __forceinline__ void bwd_drain(uint64_t* bar, uint32_t parity, uint64
 }
 
 template <int DP, bool KV>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(BwdCfg<DP, KV>::THREADS, 1)
     attn_bwd_sm100(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
                    const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
                    const __grid_constant__ CUtensorMap tm_b3, const BwdTcWork w) {
@@ -243,10 +249,11 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_p_full = bar_s_free + 2;               // [2]
   uint64_t* bar_pv_done = bar_p_full + 2;              // [2]
   uint64_t* bar_acc_done = bar_pv_done + 2;
-  uint64_t* bar_stats = bar_acc_done + 1;  // [2 warpgroups][2 slots]
+  uint64_t* bar_stats = bar_acc_done + 1;          // [NSLOT] statistics of the slot's tile written
+  uint64_t* bar_stats_free = bar_stats + C::NSLOT;  // [NSLOT] the slot's tile read by its warpgroup
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  // [2][2][BN] (LSE log2(e), D) of streamed rows (dK/dV instance); 16-byte aligned.
+  // [NSLOT][BN] (LSE log2(e), D) of streamed rows (dK/dV instance); 16-byte aligned.
   float2* s_st = reinterpret_cast<float2*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5;
@@ -268,7 +275,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar_pv_done + i, 1);
     }
     mbar_init(bar_acc_done, 3);  // one commit per issuer
-    for (int i = 0; i < 4; ++i) mbar_init(bar_stats + i, 4);
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(bar_stats + i, 4);       // the statistics warpgroup's warps
+      mbar_init(bar_stats_free + i, 4);  // the warps of the element-wise warpgroup that read it
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -295,7 +305,68 @@ __global__ void __launch_bounds__(384, 1)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // Register split (warpgroup-wide): the control warpgroup (warps 8-11) shrinks, and the
   // element-wise warpgroups grow into what it released.
-  if (warp >= 8) {
+  if (C::STATS_WG && warp >= 12) {
+    bwd_setmaxnreg_dec<C::REG_ST>();
+    // ============================================================ statistics (dK/dV instance)
+    // D = dO . O and LSE log2(e) of the 64 query rows of every streamed tile j, into slot
+    // j % NSLOT once the element-wise warpgroup that used the slot's previous tile has read it.
+    // Two threads per row, each half of the row's 16-byte chunks of the staged O and dO tiles
+    // (both tiles share one swizzled layout, so the same physical chunks pair the same elements).
+    // A row's LSE is loaded one tile ahead.
+    const int tid = threadIdx.x - 384;
+    const int sc = tid >> 1, part = tid & 1;
+    auto lse_of = [&](int gg, int tt) -> float {
+      const int qi = tt * C::BN + sc;
+      const int hq = rg.hf * w.qpk + gg;
+      return qi < w.n_q ? w.lse[(static_cast<long long>(rg.b) * w.H + hq) * w.n_q + qi] : -INFINITY;
+    };
+    int g = 0, t = rg.tb;  // head and tile of tile j
+    float lse_next = (part == 0 && rg.n > 0) ? lse_of(g, t) : 0.f;
+    bool ok = true;
+    for (int j = 0; ok && j < rg.n; ++j) {
+      const int slot = j % C::NSLOT, st = j % C::STAGES;
+      const float L = lse_next;
+      int gn = g, tn = t + 1;
+      if (tn == rg.te) {
+        tn = rg.tb;
+        ++gn;
+      }
+      if (part == 0 && j + 1 < rg.n) lse_next = lse_of(gn, tn);
+      if (j >= C::NSLOT && !(ok = bwd_wait(bar_stats_free + slot, ((j / C::NSLOT) - 1) & 1, ctl, 0x726))) break;
+      if (!(ok = bwd_wait(bar_stage_full + st, (j / C::STAGES) & 1, ctl, 0x721))) break;
+      constexpr int NCH = DP / 16;    // chunks per thread
+      constexpr int CPR = C::CB / 8;  // chunks per row of one column block
+      const uint8_t* sdo = sStage + st * C::STAGE_BYTES + C::TILE_BYTES;
+      const uint8_t* so = sdo + C::TILE_BYTES;
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int kc = part * NCH + i;
+        const int off = (kc / CPR) * C::BLK_N + sc * C::ROW_BYTES + (kc % CPR) * 16;
+        const uint4 a = *reinterpret_cast<const uint4*>(so + off);
+        const uint4 bb = *reinterpret_cast<const uint4*>(sdo + off);
+        const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
+          acc = fmaf(fx.x, fy.x, acc);
+          acc = fmaf(fx.y, fy.y, acc);
+        }
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      // Rows past the end (LSE -inf here) and empty rows get LSE log2(e) = +inf, so P = 0.
+      if (part == 0)
+        s_st[slot * C::BN + sc] = make_float2(L == -INFINITY ? INFINITY : L * 1.4426950408889634f, acc);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_stage_empty + st);  // this warp is done with the stage's O tile
+        mbar_arrive(bar_stats + slot);
+      }
+      g = gn;
+      t = tn;
+    }
+  } else if (warp >= 8) {
    bwd_setmaxnreg_dec<C::REG_CTL>();
    if (warp == 8) {
     if (lane == 0 && rg.n > 0) {
@@ -412,7 +483,6 @@ __global__ void __launch_bounds__(384, 1)
     // ==================================================================== element-wise (warps 0-7)
     const int grp = warp >> 2;  // warpgroup: streamed tiles j with j % 2 == grp
     const int row = (warp & 3) * 32 + lane;
-    const int tid = threadIdx.x & 127;  // thread within the warpgroup
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t sbuf = lane_addr + grp * C::SB_STRIDE;
     const int fixed_pos = rg.m0 + row;
@@ -438,52 +508,6 @@ __global__ void __launch_bounds__(384, 1)
       }
       row_d = acc;
     }
-    // Statistics of streamed query rows (dK/dV instance): D and LSE log2(e) of the 64 rows of the
-    // warpgroup's tile, into its slot k & 1 (k = the warpgroup's tile count).  Two threads per
-    // row, each half of the row's 16-byte chunks of the staged O and dO tiles (both tiles share
-    // one swizzled layout, so the same physical chunks pair the same elements).  A row's LSE is
-    // loaded one tile of the warpgroup ahead.
-    const int sc = tid >> 1, part = tid & 1;
-    auto lse_of = [&](int gg, int tt) -> float {
-      const int qi = tt * C::BN + sc;
-      const int hq = rg.hf * w.qpk + gg;
-      return qi < w.n_q ? w.lse[(static_cast<long long>(rg.b) * w.H + hq) * w.n_q + qi] : -INFINITY;
-    };
-    auto stats = [&](int jj, int kk, float L) -> bool {
-      const int st = jj % C::STAGES;
-      if (!bwd_wait(bar_stage_full + st, (jj / C::STAGES) & 1, ctl, 0x721)) return false;
-      constexpr int NCH = DP / 16;    // chunks per thread
-      constexpr int CPR = C::CB / 8;  // chunks per row of one column block
-      const uint8_t* sdo = sStage + st * C::STAGE_BYTES + C::TILE_BYTES;
-      const uint8_t* so = sdo + C::TILE_BYTES;
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        const int k = part * NCH + i;
-        const int off = (k / CPR) * C::BLK_N + sc * C::ROW_BYTES + (k % CPR) * 16;
-        const uint4 a = *reinterpret_cast<const uint4*>(so + off);
-        const uint4 bb = *reinterpret_cast<const uint4*>(sdo + off);
-        const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&bb);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
-          acc = fmaf(fx.x, fy.x, acc);
-          acc = fmaf(fx.y, fy.y, acc);
-        }
-      }
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      // Rows past the end (LSE -inf here) and empty rows get LSE log2(e) = +inf, so P = 0.
-      if (part == 0)
-        s_st[(grp * 2 + (kk & 1)) * C::BN + sc] =
-            make_float2(L == -INFINITY ? INFINITY : L * 1.4426950408889634f, acc);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar_stage_empty + st);  // this warp is done with the stage's O tile
-        mbar_arrive(bar_stats + grp * 2 + (kk & 1));
-      }
-      return true;
-    };
     auto advance = [&](int& gg, int& tt) {
       if (++tt == rg.te) {
         tt = rg.tb;
@@ -493,22 +517,13 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     int g = 0, t = rg.tb;  // head and tile of tile j
     if (grp == 1) advance(g, t);
-    int gn = g, tn = t;    // head and tile of tile j + 2
-    advance(gn, tn);
-    advance(gn, tn);
-    float lse_cur = (KV && part == 0 && grp < rg.n) ? lse_of(g, t) : 0.f;
     int k = 0;  // tiles of this warpgroup so far
     for (int j = grp; ok && j < rg.n; j += 2, ++k) {
       const int t0 = t * C::BN;  // first streamed row of the tile
-      float lse_next = 0.f;
-      if (KV) {
-        if (part == 0 && j + 2 < rg.n) lse_next = lse_of(gn, tn);
-        if (!(ok = stats(j, k, lse_cur))) break;
-      }
       if (!(ok = bwd_wait(bar_s_full + grp, k & 1, ctl, 0x722))) break;
-      if (KV && !(ok = bwd_wait(bar_stats + grp * 2 + (k & 1), (k >> 1) & 1, ctl, 0x723))) break;
+      if (KV && !(ok = bwd_wait(bar_stats + j % C::NSLOT, (j / C::NSLOT) & 1, ctl, 0x723))) break;
       tc_fence_after();
-      const float4* stv = reinterpret_cast<const float4*>(s_st + (grp * 2 + (k & 1)) * C::BN);
+      const float4* stv = reinterpret_cast<const float4*>(s_st + (j % C::NSLOT) * C::BN);
       uint32_t pp[32], dd[32];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -567,6 +582,11 @@ __global__ void __launch_bounds__(384, 1)
           dd[16 * h + i / 2] = bf16x2_bits(e0 * (__uint_as_float(pv[i]) - cs.y), e1 * (__uint_as_float(pv[i + 1]) - cs.w));
         }
       }
+      if (KV) {
+        // The tile's statistics are in registers: its slot may take the tile NSLOT further on.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_stats_free + j % C::NSLOT);
+      }
       // The warpgroup's P, dS columns are free once the products of its previous tile are done.
       if (k > 0 && !(ok = bwd_wait(bar_pv_done + grp, (k - 1) & 1, ctl, 0x724))) break;
       tc_fence_after();
@@ -576,11 +596,8 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p_full + grp);
-      lse_cur = lse_next;
       advance(g, t);
       advance(g, t);
-      advance(gn, tn);
-      advance(gn, tn);
     }
     // ================================================================== epilogue
     const bool have = ok && rg.n > 0 && bwd_wait(bar_acc_done, 0, ctl, 0x725);
