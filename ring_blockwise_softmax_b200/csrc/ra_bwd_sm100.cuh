@@ -530,13 +530,6 @@ __global__ void __launch_bounds__(BwdCfg<DP, KV>::THREADS, 1)
         uint32_t sv[32], pv[32];
         tmem_ld32(sbuf + C::S_COL + 32 * h, sv);
         tmem_ld32(sbuf + C::DP_COL + 32 * h, pv);
-        // The columns' (LSE log2(e), D) pairs (dK/dV instance), read from shared memory while the
-        // tensor-memory loads are in flight rather than one by one at their uses.
-        float4 cst[16];
-        if (KV) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) cst[i] = stv[16 * h + i];
-        }
         tmem_ld_wait(sv);
         reg_pin32(pv);
         if (h == 1) {
@@ -571,7 +564,7 @@ __global__ void __launch_bounds__(BwdCfg<DP, KV>::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           float4 cs = make_float4(row_l2, row_d, row_l2, row_d);  // (LSE log2(e), D) of columns i, i + 1
-          if (KV) cs = cst[i / 2];
+          if (KV) cs = stv[16 * h + i / 2];
           float e0 = bwd_ex2(fmaf(__uint_as_float(sv[i]), w.scale_log2, -cs.x));
           float e1 = bwd_ex2(fmaf(__uint_as_float(sv[i + 1]), w.scale_log2, -cs.z));
           if (masked) {
