@@ -26,14 +26,16 @@
 // S and dP here are the transposes of each other's roles in the two instances, so both use the
 // forward's operand forms unchanged.  No atomics: every gradient element has one owner.
 //
-// Roles (352 threads): two element-wise warpgroups (warps 0-3 and 4-7) take alternate streamed
-// tiles, thread = tensor-memory lane (warp % 4) * 32 + lane, all 64 columns of its row; each
-// warpgroup has its own (S, dP) buffer and P, dS columns in tensor memory, so one computes while
-// the other waits on its loads, stores and barriers.  (The dK/dV instance at DP = 128 lacks the
-// tensor memory for that and runs attn_bwd_sm100_split, further below.)  Warp 8 is the TMA
-// producer (and allocates tensor memory); warps 9 and 10 issue the MMAs: warp 9 starts S, dP of
-// tile j + 2 as soon as warpgroup j % 2 holds tile j in registers, warp 10 the products of each
-// tile once its P and dS are stored.  At the end the eight warps run the epilogue.  Every wait is
+// Roles: two element-wise warpgroups (warps 0-3 and 4-7) take alternate streamed tiles, thread =
+// tensor-memory lane (warp % 4) * 32 + lane, all 64 columns of its row; each warpgroup has its
+// own (S, dP) buffer and P, dS columns in tensor memory, so one computes while the other waits on
+// its loads, stores and barriers.  (The dK/dV instance at DP = 128 lacks the tensor memory for
+// that and runs attn_bwd_sm100_split, further below.)  Warp 8 is the TMA producer (and allocates
+// tensor memory); warps 9, 10 and 11 issue the MMAs: S and dP of tile j + 2 (warps 9, 10) as soon
+// as warpgroup j % 2 holds tile j in registers, the products of each tile (warp 11) once its P
+// and dS are stored.  The dK/dV instance adds warps 12-15, which compute the streamed rows' LSE
+// and D a few tiles ahead into shared-memory slots.  Registers are rebalanced with setmaxnreg
+// (BwdCfg::REG_*).  At the end the eight element-wise warps run the epilogue.  Every wait is
 // bounded.
 #pragma once
 
