@@ -337,7 +337,7 @@ def config_dict(w, args):
         name += f", {w.layout} shards instead"
     return {"workload": f"cfg{w.cfg}: {name}", "B": w.B, "H": w.H, "H_kv": w.H_kv or w.H, "N": w.N, "d": w.d,
             "causal": w.causal, "window": w.window,
-            "P": w.P, "layout": w.layout, "schedule": args.schedule,
+            "P": w.P, "layout": w.layout, "schedule": args.schedule, "striped_walk": args.striped_walk,
             "l2": "flushed between timed steps (256 MiB write outside the events)",
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
 
@@ -398,8 +398,18 @@ def forward_roofline(w, ms: float, world: int, peak: float, peak_kind: str, laun
                  f"step's {launches} serialised launches (CUDA events on the launch stream)")}
 
 
-def traffic_key(w, backward: bool = False) -> str:
+def traffic_key(w, backward: bool = False, walk: str = "shard") -> str:
+    """Key of a workload's recorded DRAM traffic: the configuration plus every override that
+    changes what the attention kernel reads (reduced lengths are never recorded)."""
+    from ring_blockwise_softmax_b200 import inputs as I
+
     key = f"cfg{w.cfg}" + ("" if w.H_kv is None else f"-kv{w.H_kv}") + ("" if w.window is None else f"-w{w.window}")
+    if w.layout != I.WORKLOADS[w.cfg].layout:
+        key += f"-{w.layout}"
+    if w.N != I.WORKLOADS[w.cfg].N:
+        key += f"-n{w.N}"
+    if walk != "shard" and w.layout == "striped" and w.d > 64:
+        key += f"-{walk}walk"
     return key + ("-bwd" if backward else "")
 
 
@@ -571,7 +581,7 @@ def run_gpu(args, w):
             del bufs_c
             torch.cuda.empty_cache()
             v_c, roof_c = forward_roofline(wc, ms_c, world, peak, peak_kind, l_c,
-                                           recorded_traffic(traffic_key(wc), args.schedule))
+                                           recorded_traffic(traffic_key(wc, walk=args.striped_walk), args.schedule))
             others[f"cfg{c}"] = {
                 "workload": wc.name, "steps": steps_c, "ms_per_step": ms_c, "value": v_c, "unit": "TFLOP/s",
                 "flops_per_step": wc.flops(), "pct_of_spec_bf16_peak": 100.0 * (v_c / world) / SPEC_BF16_TFLOPS,
@@ -591,7 +601,7 @@ def run_gpu(args, w):
     else:
         _, roof = forward_roofline(w, ms, world, peak, peak_kind, launches_per_step,
                                    args.traffic if args.traffic is not None
-                                   else recorded_traffic(traffic_key(w), args.schedule))
+                                   else recorded_traffic(traffic_key(w, walk=args.striped_walk), args.schedule))
     line = {
         "metric": METRIC_BWD if args.backward else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps,
@@ -650,6 +660,8 @@ def main(argv=None):
                     help="grouped-query variant of the workload: K and V with this many heads (must divide H)")
     ap.add_argument("--layout", choices=["contiguous", "striped"], default=None,
                     help="ring shard layout override (the workload's own by default)")
+    ap.add_argument("--striped-walk", choices=["shard", "tile"], default="shard",
+                    help="K/V walk order of fused rings over striped shards (ra_set_striped_walk)")
     ap.add_argument("--n", type=int, default=None,
                     help="sequence length override: a smaller case of the workload's layout (profiling)")
     ap.add_argument("--traffic", type=float, default=None,
@@ -658,6 +670,11 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from ring_blockwise_softmax_b200 import inputs as I
+
+    if args.striped_walk != "shard" and args.impl != "reference":
+        from ring_blockwise_softmax_b200 import ra_attn as ra_walk
+
+        ra_walk.set_striped_walk(args.striped_walk)
 
     w = I.WORKLOADS[args.config]
     if args.layout is not None:

@@ -52,13 +52,11 @@ namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
 constexpr double kLog2e = 1.4426950408889634;
-#ifndef RA_TILE_MAJOR
-#define RA_TILE_MAJOR 0
-#endif
-// 1: multi-step launches over striped shards walk K/V tile index first, the shards inside.  That
-// order reads 3.4x fewer DRAM bytes on a striped d = 128 ring (1.8 instead of 6.7 GB at B=1 H=32
-// N=32768 P=8) but runs 2.7 % slower under the power cap, so the shard-major walk is the default.
-constexpr bool kTileMajor = RA_TILE_MAJOR != 0;
+// Walk order of multi-step launches over striped shards (ra_set_striped_walk): 1 = K/V tile
+// index first, the shards inside.  That order reads 3.4x fewer DRAM bytes on a striped d = 128
+// ring (1.8 instead of 6.7 GB at B=1 H=32 N=32768 P=8) but runs 2.7 % slower under the power cap,
+// so the shard-major walk is the default.
+std::atomic<int> g_striped_walk{RA_WALK_SHARD_MAJOR};
 
 thread_local std::string t_last_error;
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
@@ -714,7 +712,7 @@ static ra_status_t ring_fwd_impl(const ra_tensor_t* q, const ra_tensor_t* k, con
   w.k_sstep = shard_rows;
   w.k_ustride = tok_rows;
   w.r_major = striped ? 0 : 1;
-  w.tile_major = striped && kTileMajor ? 1 : 0;
+  w.tile_major = striped && g_striped_walk.load() == RA_WALK_TILE_MAJOR ? 1 : 0;
   set_operand_ptrs(w, q, k, v, shard_rows, tok_rows);
   w.o = o->data;
   w.o_sb = o->stride[0];
@@ -1151,6 +1149,13 @@ ra_status_t ra_get_device_status(ra_stream_t stream) {
 ra_status_t ra_set_wait_timeout_ns(uint64_t ns) {
   if (ns < 1000 || ns > 60ull * 1000000000ull) return fail(RA_ERR_INVALID_ARG, "timeout must be in [1 us, 60 s]");
   g_wait_limit_ns.store(ns);
+  return ok();
+}
+
+ra_status_t ra_set_striped_walk(int order) {
+  if (order != RA_WALK_SHARD_MAJOR && order != RA_WALK_TILE_MAJOR)
+    return fail(RA_ERR_INVALID_ARG, "walk order must be RA_WALK_SHARD_MAJOR or RA_WALK_TILE_MAJOR");
+  g_striped_walk.store(order);
   return ok();
 }
 

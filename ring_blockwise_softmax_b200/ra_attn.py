@@ -42,7 +42,7 @@ SCHEDULES = {"stepwise": RA_RING_STEPWISE, "fused": RA_RING_FUSED}
 # Exported symbols of the library, in header order (the CPU test checks each one is present).
 SYMBOLS = (
     "ra_attn_fwd", "ra_attn_fwd_window", "ra_attn_bwd", "ra_attn_partial", "ra_lse_merge", "ra_lse_merge_n", "ra_ring_workspace_size",
-    "ra_ring_fwd", "ra_ring_fwd_window", "ra_ring_fwd_host", "ra_ring_fwd_noalloc", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_debug_unarrived_wait",
+    "ra_ring_fwd", "ra_ring_fwd_window", "ra_ring_fwd_host", "ra_ring_fwd_noalloc", "ra_get_device_status", "ra_set_wait_timeout_ns", "ra_set_striped_walk", "ra_debug_unarrived_wait",
     "ra_debug_exp2", "ra_status_string", "ra_last_error", "ra_version",
 )
 
@@ -79,6 +79,7 @@ _lib.ra_ring_fwd_noalloc.argtypes = [_T, _T, _T, ctypes.c_int, ctypes.c_int, cty
                                      _S]
 _lib.ra_get_device_status.argtypes = [_S]
 _lib.ra_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+_lib.ra_set_striped_walk.argtypes = [ctypes.c_int]
 _lib.ra_debug_unarrived_wait.argtypes = [ctypes.c_uint64, _S]
 _lib.ra_debug_exp2.argtypes = [_F, _F, _F, ctypes.c_int64, _S]
 _lib.ra_status_string.argtypes = [ctypes.c_int]
@@ -285,6 +286,14 @@ def get_device_status(stream=None) -> int:
 
 def set_wait_timeout_ns(ns: int):
     _check(_lib.ra_set_wait_timeout_ns(int(ns)), "ra_set_wait_timeout_ns")
+
+
+WALKS = {"shard": 0, "tile": 1}  # RA_WALK_SHARD_MAJOR, RA_WALK_TILE_MAJOR
+
+
+def set_striped_walk(order: str):
+    """ra_set_striped_walk: "shard" (default) or "tile", the K/V walk of fused rings over striped shards."""
+    _check(_lib.ra_set_striped_walk(WALKS[order]), "ra_set_striped_walk")
 
 
 def debug_unarrived_wait(timeout_ns: int, stream=None):

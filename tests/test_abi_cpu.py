@@ -100,6 +100,11 @@ def test_host_validation_without_a_device(ra):
     assert lib.ra_lse_merge_n(None, None, 33, None, None, 10, 64, None) == ra.RA_ERR_INVALID_ARG
     # timeout limits
     assert lib.ra_set_wait_timeout_ns(10) == ra.RA_ERR_INVALID_ARG
+    # walk order over striped shards: the two named orders only (a process-wide setting, restored)
+    assert lib.ra_set_striped_walk(2) == ra.RA_ERR_INVALID_ARG
+    assert lib.ra_set_striped_walk(-1) == ra.RA_ERR_INVALID_ARG
+    assert lib.ra_set_striped_walk(1) == ra.RA_OK
+    assert lib.ra_set_striped_walk(0) == ra.RA_OK
 
 
 def test_ring_workspace_size(ra):

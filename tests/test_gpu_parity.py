@@ -164,16 +164,41 @@ def test_lse_merge_n(ra, d, k):
 @pytest.mark.parametrize("P,N", [(2, 600), (3, 384), (8, 1000), (16, 1040)])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("schedule", ["stepwise", "fused"])
-def test_ring_striped_d128(ra, P, N, causal, schedule):
-    """Striped rings at d = 128, whose fused launches walk K/V tile index first and the shards
-    inside (shards of 300, 128, 125 and 65 rows: ragged 64-key tiles in every shard)."""
+@pytest.mark.parametrize("walk", ["shard", "tile"])
+def test_ring_striped_d128(ra, P, N, causal, schedule, walk):
+    """Striped rings at d = 128 with either walk order of the fused launches over the shards'
+    K/V tiles (shards of 300, 128, 125 and 65 rows: ragged 64-key tiles in every shard)."""
     q, k, v = I.make_small(1, 2, N, 128, "bf16", seed=31 * P + N)
     qd, kd, vd = _dev(q, k, v)
-    o, lse = ra.ring_attention(qd, kd, vd, P, "striped", causal, schedule=schedule)
-    torch.cuda.synchronize()
+    ra.set_striped_walk(walk)
+    try:
+        o, lse = ra.ring_attention(qd, kd, vd, P, "striped", causal, schedule=schedule)
+        torch.cuda.synchronize()
+    finally:
+        ra.set_striped_walk("shard")
     assert ra.get_device_status() == ra.RA_OK
     o_ref, l_ref = oracle_heads(to64(q), to64(k), to64(v), 1 / math.sqrt(128), causal)
-    compare(to64(o), to64(lse), o_ref, l_ref, "bf16", f"striped d=128 P={P} causal={causal} {schedule}")
+    compare(to64(o), to64(lse), o_ref, l_ref, "bf16", f"striped d=128 P={P} causal={causal} {schedule} {walk}")
+
+
+@pytest.mark.parametrize("window", [1, 100, 300, 5000])
+def test_ring_striped_tile_walk_window(ra, window):
+    """The tile-major walk's division-free bounds with a sliding window (the first visible key of
+    every shard), striped d = 128, fused schedule, P = 8 over 1000 tokens."""
+    q, k, v = I.make_small(1, 2, 1000, 128, "bf16", seed=4000 + window, v_dist="uniform")
+    qd, kd, vd = _dev(q, k, v)
+    outs = {}
+    for walk in ("shard", "tile"):
+        ra.set_striped_walk(walk)
+        try:
+            outs[walk] = ra.ring_attention(qd, kd, vd, 8, "striped", True, schedule="fused", window=window)
+            torch.cuda.synchronize()
+        finally:
+            ra.set_striped_walk("shard")
+        assert ra.get_device_status() == ra.RA_OK
+    o_ref, l_ref = oracle_heads(to64(q), to64(k), to64(v), 1 / math.sqrt(128), True, window=window)
+    for walk, (o, lse) in outs.items():
+        compare(to64(o), to64(lse), o_ref, l_ref, "bf16", f"striped window={window} {walk}")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
