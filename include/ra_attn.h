@@ -284,7 +284,7 @@ ra_status_t ra_set_wait_timeout_ns(uint64_t ns);
  * Striped shards interleave their keys in memory (key u of shard s sits at position u * P + s),
  * so the tile-major order reads each stretch of K/V once per work item instead of once per shard:
  * on one B200, B=1 H=32 N=32768 d=128 P=8 causal reads 1.8 instead of 6.7 GB of DRAM per launch,
- * but runs about 2.7 % slower.  Either order visits the same tiles (results equal within
+ * but runs 2-3 % slower.  Either order visits the same tiles (results equal within
  * rounding).  Contiguous shards, other head dims and one-step launches ignore the setting.
  * Process-wide; applies to later calls.  Returns RA_ERR_INVALID_ARG for any other value. */
 #define RA_WALK_SHARD_MAJOR 0
