@@ -262,7 +262,6 @@ __global__ void __launch_bounds__(BwdCfg<DP, KV>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   WaitCtl ctl{abort_flag, w.wait_limit_ns, w.dev_status};
   const BwdRange rg = bwd_range<KV>(w);
-  const int nt = rg.te - rg.tb;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_fixed, 1);
@@ -726,7 +725,6 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = threadIdx.x & 31;
   WaitCtl ctl{abort_flag, w.wait_limit_ns, w.dev_status};
   const BwdRange rg = bwd_range<KV>(w);
-  const int nt = rg.te - rg.tb;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_fixed, 1);
