@@ -51,3 +51,34 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
     with redirect_stdout(buf):
         rc = bench.main(["--impl", "reference", "--gpus", "2", "--config", "1", "--steps", "1", "--warmup", "3"])
     assert rc == 0 and buf.getvalue().strip() == ""
+
+
+def test_recorded_traffic_only_for_the_captured_launch():
+    """The roofline's DRAM traffic comes from a capture of the same kernel sources on the same
+    launch: a layout or length override, or the other walk order over striped shards, must not
+    pick up the default launch's figure (and the tile walk must find its own)."""
+    sys.path.insert(0, ROOT)
+    import dataclasses
+
+    import bench
+    from ring_blockwise_softmax_b200 import inputs as I
+
+    w3 = I.WORKLOADS[3]  # striped, d = 128
+    keys = {
+        bench.traffic_key(w3),
+        bench.traffic_key(w3, walk="tile"),
+        bench.traffic_key(dataclasses.replace(w3, layout="contiguous")),
+        bench.traffic_key(dataclasses.replace(w3, N=w3.N // 4)),
+        bench.traffic_key(w3, backward=True),
+    }
+    assert len(keys) == 5
+    assert bench.traffic_key(w3) == "cfg3"
+    # the walk order only matters for striped shards at d > 64
+    w2 = I.WORKLOADS[2]
+    assert bench.traffic_key(w2, walk="tile") == bench.traffic_key(w2)
+    rec = json.load(open(os.path.join(ROOT, "profiles", "fmha_traffic.json")))
+    if rec["kernel_sources_sha256"] == bench.kernel_sources_hash():
+        assert bench.recorded_traffic(bench.traffic_key(w3), "fused") is not None
+        assert bench.recorded_traffic(bench.traffic_key(w3, walk="tile"), "fused") is not None
+        assert bench.recorded_traffic(bench.traffic_key(dataclasses.replace(w3, layout="contiguous")), "fused") is None
+        assert bench.recorded_traffic(bench.traffic_key(w3), "stepwise") is None
